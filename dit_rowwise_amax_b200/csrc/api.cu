@@ -1,0 +1,436 @@
+// C-ABI entry points of libfp8dit (declared and documented in include/fp8dit.h):
+// argument validation, per-device state, TMA descriptors, the tile plan bound
+// at layer creation, and dispatch to the kernels. Nothing here computes on
+// the host: every step of the path runs in the CUDA kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "fp8dit_internal.cuh"
+
+// Per-device error word raised by expired bounded waits.
+__device__ uint32_t g_fp8dit_error_word;
+
+namespace fp8dit {
+
+// ------------------------------------------------------------------ errors
+static thread_local char t_last_error[512];
+
+void set_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+    va_end(ap);
+}
+
+fp8dit_status cuda_fail(cudaError_t e, const char* what) {
+    set_error("%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+    return FP8DIT_ERR_CUDA;
+}
+
+static fp8dit_status invalid(const char* msg) {
+    set_error("invalid argument: %s", msg);
+    return FP8DIT_ERR_INVALID_ARG;
+}
+
+static fp8dit_status unsupported(const char* msg) {
+    set_error("unsupported shape: %s", msg);
+    return FP8DIT_ERR_UNSUPPORTED_SHAPE;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------- devices
+constexpr int kMaxDevices = 64;
+static DeviceInfo g_dev[kMaxDevices];
+static bool g_dev_ready[kMaxDevices];
+static std::mutex g_dev_mutex;
+
+const DeviceInfo* device_info() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cuda_fail(e, "cudaGetDevice");
+        return nullptr;
+    }
+    if (dev < 0 || dev >= kMaxDevices) {
+        set_error("device ordinal %d beyond %d", dev, kMaxDevices);
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_dev_ready[dev]) {
+        DeviceInfo info{};
+        int major = 0, minor = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&info.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+                cudaSuccess) {
+            cuda_fail(e, "cudaDeviceGetAttribute");
+            return nullptr;
+        }
+        if (major != 10 || minor != 0) {
+            set_error("device %d is sm_%d%d; this library is built for sm_100a only", dev, major, minor);
+            return nullptr;
+        }
+        void* word = nullptr;
+        if ((e = cudaGetSymbolAddress(&word, g_fp8dit_error_word)) != cudaSuccess) {
+            cuda_fail(e, "cudaGetSymbolAddress(error word)");
+            return nullptr;
+        }
+        info.err_word = static_cast<uint32_t*>(word);
+        g_dev[dev] = info;
+        g_dev_ready[dev] = true;
+    }
+    return &g_dev[dev];
+}
+
+static DevErr dev_err(const DeviceInfo* d) { return DevErr{d->err_word, kDefaultWaitLimitNs}; }
+
+// ------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+fp8dit_status encode_tma_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        set_error("cuTensorMapEncodeTiled is not available from the driver");
+        return FP8DIT_ERR_CUDA;
+    }
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (CUresult %d) for %llu x %llu", (int)r, (unsigned long long)outer,
+                  (unsigned long long)inner);
+        return FP8DIT_ERR_CUDA;
+    }
+    return FP8DIT_OK;
+}
+
+// ------------------------------------------------------------- self test
+namespace {
+__global__ void selftest_wait_kernel(DevErr err) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbarrier_init();
+        // Nothing ever arrives: the bounded wait must expire and report.
+        mbar_wait_bounded(&bar, 0, nullptr, err);
+    }
+}
+}  // namespace
+
+cudaError_t launch_selftest_wait(cudaStream_t stream, DevErr err) {
+    selftest_wait_kernel<<<1, 32, 0, stream>>>(err);
+    return cudaGetLastError();
+}
+
+}  // namespace fp8dit
+
+using namespace fp8dit;
+
+// ------------------------------------------------------------- linear handle
+struct fp8dit_linear_s {
+    int64_t N, K;
+    const uint8_t* qw;
+    const float* sw;
+    const uint16_t* bias;
+    int device;
+    int num_sms;
+    CUtensorMap tmB[kNumCfgs];  // weight descriptors, one per tile configuration
+};
+
+// Tile plan: 128 x 256 tiles unless they leave more than half the SMs idle,
+// then 128 x 128. Depends only on (M, N, n_problems, SM count).
+static int choose_cfg(const fp8dit_linear_s* h, int64_t M, int n_problems) {
+    const int64_t tm = (M + kGemmBlockM - 1) / kGemmBlockM;
+    const int64_t tiles256 = tm * ((h->N + 255) / 256) * n_problems;
+    return tiles256 * 2 >= h->num_sms ? kCfg128x256 : kCfg128x128;
+}
+
+static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, const uint8_t* qa, const float* sa,
+                              uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev) {
+    const int cfg = choose_cfg(hs[0], M, n);
+    const int bn = gemm_block_n(cfg);
+    GemmArgs args;
+    memset(&args, 0, sizeof(args));
+    fp8dit_status st = encode_tma_2d_u8(&args.tmA, qa, (uint64_t)hs[0]->K, (uint64_t)M, (uint64_t)hs[0]->K,
+                                        kGemmBlockK, kGemmBlockM, true);
+    if (st != FP8DIT_OK) return st;
+    const int tiles_m = (int)((M + kGemmBlockM - 1) / kGemmBlockM);
+    int tiles = 0;
+    for (int g = 0; g < n; ++g) {
+        args.tmB[g] = hs[g]->tmB[cfg];
+        GemmProblem& p = args.prob[g];
+        p.sw = hs[g]->sw;
+        p.bias = hs[g]->bias;
+        p.y = ys[g];
+        p.N = (int32_t)hs[g]->N;
+        p.tiles_n = (int32_t)((hs[g]->N + bn - 1) / bn);
+        p.tile_start = tiles;
+        tiles += tiles_m * p.tiles_n;
+    }
+    args.sa = sa;
+    args.M = (int32_t)M;
+    args.K = (int32_t)hs[0]->K;
+    args.G = n;
+    args.tiles_m = tiles_m;
+    args.num_tiles = tiles;
+    args.num_kb = (int32_t)((hs[0]->K + kGemmBlockK - 1) / kGemmBlockK);
+    args.err = dev_err(dev);
+    cudaError_t e = launch_gemm(cfg, args, gemm_ctas_for(cfg, tiles, dev), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "FP8 GEMM launch");
+    return FP8DIT_OK;
+}
+
+// Largest sizes the kernels index with 32-bit tile / row arithmetic.
+constexpr int64_t kMaxRows = (int64_t)1 << 30;
+constexpr int64_t kMaxK = (int64_t)1 << 20;
+
+extern "C" {
+
+const char* fp8dit_last_error_string(void) { return t_last_error; }
+
+fp8dit_status fp8_quantize_rowwise(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, fp8dit_format fmt,
+                                   uint8_t* q, int64_t ldq, float* scale, fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (fmt != FP8DIT_E4M3FN && fmt != FP8DIT_E5M2) return invalid("format");
+    if (M < 0 || K <= 0) return invalid("M must be >= 0 and K > 0");
+    if (K % 16 != 0) return unsupported("K must be a multiple of 16");
+    if (ldx < K || ldx % 8 != 0) return invalid("ldx must be >= K and a multiple of 8");
+    if (ldq < K || ldq % 16 != 0) return invalid("ldq must be >= K and a multiple of 16");
+    if (M > kMaxRows || K > kMaxK) return unsupported("M or K too large");
+    if (M == 0) return FP8DIT_OK;
+    if (!x || !q || !scale) return invalid("null pointer");
+    if (!aligned16(x) || !aligned16(q)) return invalid("x and q must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(scale) & 3u) return invalid("scale must be 4-byte aligned");
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    cudaError_t e = launch_quantize_rows(x, M, K, ldx, fmt, q, ldq, scale, (cudaStream_t)stream, dev);
+    return e == cudaSuccess ? FP8DIT_OK : cuda_fail(e, "rowwise quantise launch");
+}
+
+fp8dit_status fp8_quantize_weight_per_channel(const uint16_t* w, int64_t N, int64_t K, fp8dit_format fmt,
+                                              uint8_t* qw, float* sw, fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (N <= 0) return invalid("N must be > 0");
+    return fp8_quantize_rowwise(w, N, K, K, fmt, qw, K, sw, stream);
+}
+
+size_t fp8_quantize_weight_per_tensor_workspace_size(int32_t n_tensors) {
+    return per_tensor_workspace_bytes(n_tensors);
+}
+
+fp8dit_status fp8_quantize_weight_per_tensor(const fp8dit_tensor_desc* tensors, int32_t n_tensors,
+                                             fp8dit_format fmt, void* workspace, size_t ws_bytes,
+                                             fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (n_tensors < 0) return invalid("n_tensors must be >= 0");
+    if (n_tensors == 0 || tensors == nullptr) {
+        set_error("invalid input: no tensors to convert");
+        return FP8DIT_ERR_EMPTY;
+    }
+    if (fmt != FP8DIT_E4M3FN && fmt != FP8DIT_E5M2) return invalid("format");
+    int64_t total = 0;
+    for (int32_t i = 0; i < n_tensors; ++i) {
+        const fp8dit_tensor_desc& d = tensors[i];
+        if (d.numel < 0) return invalid("numel must be >= 0");
+        if (d.numel == 0) continue;
+        if (d.numel > ((int64_t)1 << 40)) return unsupported("tensor too large");
+        if (!d.src || !d.dst || !d.scale) return invalid("null pointer in tensor descriptor");
+        if (!aligned16(d.src) || !aligned16(d.dst)) return invalid("src and dst must be 16-byte aligned");
+        if (reinterpret_cast<uintptr_t>(d.scale) & 3u) return invalid("scale must be 4-byte aligned");
+        total += d.numel;
+    }
+    if (total == 0) {
+        set_error("no tensor converted to %s: every tensor is empty", fmt == FP8DIT_E4M3FN ? "float8_e4m3fn"
+                                                                                             : "float8_e5m2");
+        return FP8DIT_ERR_EMPTY;
+    }
+    if (!workspace || !aligned16(workspace)) return invalid("workspace must be non-null and 16-byte aligned");
+    if (ws_bytes < per_tensor_workspace_bytes(n_tensors)) return invalid("workspace too small");
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    cudaError_t e = launch_per_tensor(tensors, n_tensors, fmt, workspace, (cudaStream_t)stream, dev, dev_err(dev));
+    return e == cudaSuccess ? FP8DIT_OK : cuda_fail(e, "per-tensor conversion launch");
+}
+
+fp8dit_status fp8_linear_create(int64_t N, int64_t K, const uint8_t* qw, const float* sw, const uint16_t* bias,
+                                int device, fp8dit_linear* out) {
+    t_last_error[0] = 0;
+    if (!out) return invalid("out is null");
+    *out = nullptr;
+    if (N <= 0 || K <= 0) return invalid("N and K must be > 0");
+    if (N % 8 != 0) return unsupported("N must be a multiple of 8");
+    if (K % 16 != 0) return unsupported("K must be a multiple of 16");
+    if (N > kMaxRows || K > kMaxK) return unsupported("N or K too large");
+    if (!qw || !sw) return invalid("qw and sw must be non-null");
+    if (!aligned16(qw) || !aligned16(sw)) return invalid("qw and sw must be 16-byte aligned");
+    if (bias && !aligned16(bias)) return invalid("bias must be 16-byte aligned");
+    int prev = 0;
+    cudaError_t e = cudaGetDevice(&prev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (device != prev && (e = cudaSetDevice(device)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    fp8dit_status st = FP8DIT_OK;
+    fp8dit_linear_s* h = nullptr;
+    const DeviceInfo* dev = device_info();
+    if (!dev) {
+        st = FP8DIT_ERR_CUDA;
+    } else {
+        h = new fp8dit_linear_s();
+        h->N = N;
+        h->K = K;
+        h->qw = qw;
+        h->sw = sw;
+        h->bias = bias;
+        h->device = device;
+        h->num_sms = dev->num_sms;
+        for (int cfg = 0; cfg < kNumCfgs && st == FP8DIT_OK; ++cfg)
+            st = encode_tma_2d_u8(&h->tmB[cfg], qw, (uint64_t)K, (uint64_t)N, (uint64_t)K, kGemmBlockK,
+                                  (uint32_t)gemm_block_n(cfg), true);
+    }
+    if (device != prev) cudaSetDevice(prev);
+    if (st != FP8DIT_OK) {
+        delete h;
+        return st;
+    }
+    *out = h;
+    return FP8DIT_OK;
+}
+
+fp8dit_status fp8_linear_destroy(fp8dit_linear h) {
+    t_last_error[0] = 0;
+    delete h;
+    return FP8DIT_OK;
+}
+
+static fp8dit_status check_device(const fp8dit_linear_s* h) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev != h->device) return invalid("current device differs from the layer's device");
+    return FP8DIT_OK;
+}
+
+fp8dit_status fp8_scaled_linear(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, const uint8_t* qa,
+                                const float* sa, uint8_t* qa_scratch, float* sa_scratch, uint16_t* y,
+                                fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (!h) return invalid("null handle");
+    if (M < 0) return invalid("M must be >= 0");
+    if (M > kMaxRows) return unsupported("M too large");
+    if (M == 0) return FP8DIT_OK;
+    if (!y || !aligned16(y)) return invalid("y must be non-null and 16-byte aligned");
+    if (a_bf16) {
+        if (qa || sa) return invalid("pass either a_bf16 or (qa, sa), not both");
+        if (!qa_scratch || !sa_scratch) return invalid("a_bf16 needs qa_scratch and sa_scratch");
+        if (!aligned16(a_bf16) || !aligned16(qa_scratch)) return invalid("a_bf16 and qa_scratch must be 16-byte aligned");
+        if (reinterpret_cast<uintptr_t>(sa_scratch) & 3u) return invalid("sa_scratch must be 4-byte aligned");
+    } else {
+        if (!qa || !sa) return invalid("pass a_bf16, or both qa and sa");
+        if (!aligned16(qa)) return invalid("qa must be 16-byte aligned");
+        if (reinterpret_cast<uintptr_t>(sa) & 3u) return invalid("sa must be 4-byte aligned");
+    }
+    fp8dit_status st = check_device(h);
+    if (st != FP8DIT_OK) return st;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    if (a_bf16) {
+        cudaError_t e = launch_quantize_rows(a_bf16, M, h->K, h->K, FP8DIT_E4M3FN, qa_scratch, h->K, sa_scratch,
+                                             (cudaStream_t)stream, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "activation quantise launch");
+        qa = qa_scratch;
+        sa = sa_scratch;
+    }
+    return run_gemm(&h, 1, M, qa, sa, &y, (cudaStream_t)stream, dev);
+}
+
+fp8dit_status fp8_scaled_linear_multi(const fp8dit_linear* hs, int32_t n, int64_t M, const uint16_t* a_bf16,
+                                      uint8_t* qa_scratch, float* sa_scratch, uint16_t* const* ys,
+                                      fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (!hs || !ys) return invalid("hs and ys must be non-null");
+    if (n < 1 || n > kMaxGroups) return invalid("n must be in 1..4");
+    for (int32_t i = 0; i < n; ++i) {
+        if (!hs[i]) return invalid("null handle");
+        if (hs[i]->K != hs[0]->K || hs[i]->device != hs[0]->device) return invalid("handles differ in K or device");
+        if (!ys[i] || !aligned16(ys[i])) return invalid("each ys[i] must be non-null and 16-byte aligned");
+    }
+    if (M < 0) return invalid("M must be >= 0");
+    if (M > kMaxRows) return unsupported("M too large");
+    if (M == 0) return FP8DIT_OK;
+    if (!a_bf16 || !qa_scratch || !sa_scratch) return invalid("a_bf16, qa_scratch and sa_scratch are required");
+    if (!aligned16(a_bf16) || !aligned16(qa_scratch)) return invalid("a_bf16 and qa_scratch must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(sa_scratch) & 3u) return invalid("sa_scratch must be 4-byte aligned");
+    fp8dit_status st = check_device(hs[0]);
+    if (st != FP8DIT_OK) return st;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    cudaError_t e = launch_quantize_rows(a_bf16, M, hs[0]->K, hs[0]->K, FP8DIT_E4M3FN, qa_scratch, hs[0]->K,
+                                         sa_scratch, (cudaStream_t)stream, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "activation quantise launch");
+    return run_gemm(hs, n, M, qa_scratch, sa_scratch, ys, (cudaStream_t)stream, dev);
+}
+
+fp8dit_status fp8_linear_plan(fp8dit_linear h, int64_t M, int32_t n_problems, int32_t* block_m, int32_t* block_n,
+                              int32_t* ctas) {
+    t_last_error[0] = 0;
+    if (!h || M < 0 || n_problems < 1 || n_problems > kMaxGroups) return invalid("plan arguments");
+    const int cfg = choose_cfg(h, M, n_problems);
+    const int bn = gemm_block_n(cfg);
+    const int64_t tiles = ((M + kGemmBlockM - 1) / kGemmBlockM) * ((h->N + bn - 1) / bn) * n_problems;
+    if (block_m) *block_m = kGemmBlockM;
+    if (block_n) *block_n = bn;
+    if (ctas) *ctas = (int32_t)(tiles < h->num_sms ? tiles : h->num_sms);
+    return FP8DIT_OK;
+}
+
+fp8dit_status fp8dit_device_error(fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    uint32_t word = 0;
+    if ((e = cudaMemcpy(&word, dev->err_word, sizeof(word), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "reading the device error word");
+    if (word != 0) {
+        if ((e = cudaMemset(dev->err_word, 0, sizeof(word))) != cudaSuccess)
+            return cuda_fail(e, "clearing the device error word");
+        set_error("a bounded device wait expired (error word 0x%x)", word);
+        return FP8DIT_ERR_TIMEOUT;
+    }
+    return FP8DIT_OK;
+}
+
+fp8dit_status fp8dit_selftest_expired_wait(int64_t limit_ns, fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (limit_ns < 1000 || limit_ns > 10000000000ll) return invalid("limit_ns must be in 1e3 .. 1e10");
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    cudaError_t e = launch_selftest_wait((cudaStream_t)stream, DevErr{dev->err_word, (unsigned long long)limit_ns});
+    return e == cudaSuccess ? FP8DIT_OK : cuda_fail(e, "self-test launch");
+}
+
+}  // extern "C"

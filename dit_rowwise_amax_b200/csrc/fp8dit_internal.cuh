@@ -1,0 +1,259 @@
+// Internal declarations and sm_100a device helpers shared by the fp8dit
+// kernels: mbarriers, TMA (no multicast anywhere), tcgen05 / TMEM, and the
+// bounded wait every spin in the library goes through.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fp8dit.h"
+
+namespace fp8dit {
+
+// ------------------------------------------------------------------ errors
+// Bits of the per-device error word.
+enum : uint32_t {
+    kDevErrTimeout = 1u,
+};
+
+// Where a kernel reports an expired wait, and how long a wait may last.
+struct DevErr {
+    uint32_t* word;
+    unsigned long long limit_ns;
+};
+
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+
+// ------------------------------------------------------------- host side
+// Per-device facts, fetched once per device.
+struct DeviceInfo {
+    int num_sms;
+    int max_smem_optin;
+    uint32_t* err_word;  // device address of the library's error word
+};
+
+// Returns nullptr (and sets the last error) on failure. Uses the current device.
+const DeviceInfo* device_info();
+void set_error(const char* fmt, ...);
+fp8dit_status cuda_fail(cudaError_t e, const char* what);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+fp8dit_status encode_tma_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                               bool swizzle128);
+
+// Launchers (each validates nothing; the API layer has done it).
+cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int fmt,
+                                 uint8_t* q, int64_t ldq, float* scale, cudaStream_t stream,
+                                 const DeviceInfo* dev);
+
+struct PerTensorDevDesc {
+    const uint16_t* src;
+    int64_t numel;
+    uint8_t* dst;
+    float* scale;
+};
+size_t per_tensor_workspace_bytes(int32_t n);
+cudaError_t launch_per_tensor(const fp8dit_tensor_desc* host_descs, int32_t n, int fmt, void* ws,
+                              cudaStream_t stream, const DeviceInfo* dev, DevErr err);
+
+cudaError_t launch_selftest_wait(cudaStream_t stream, DevErr err);
+
+// Grouped GEMM: up to kMaxGroups products sharing the quantised A.
+constexpr int kMaxGroups = 4;
+
+struct GemmProblem {
+    const float* sw;
+    const uint16_t* bias;  // may be null
+    uint16_t* y;
+    int32_t N;
+    int32_t tiles_n;
+    int32_t tile_start;  // first global tile index of this problem
+};
+
+struct alignas(64) GemmArgs {
+    CUtensorMap tmA;
+    CUtensorMap tmB[kMaxGroups];
+    GemmProblem prob[kMaxGroups];
+    const float* sa;
+    int32_t M, K, G;
+    int32_t tiles_m;
+    int32_t num_tiles;
+    int32_t num_kb;
+    DevErr err;
+};
+
+// Tile configurations the plan chooses from.
+enum GemmConfig : int32_t {
+    kCfg128x256 = 0,
+    kCfg128x128 = 1,
+    kNumCfgs = 2,
+};
+int gemm_block_n(int cfg);
+constexpr int kGemmBlockM = 128;
+constexpr int kGemmBlockK = 128;  // bytes = FP8 elements per k-block (one 128 B swizzle row)
+
+cudaError_t launch_gemm(int cfg, const GemmArgs& args, int ctas, cudaStream_t stream);
+int gemm_ctas_for(int cfg, int num_tiles, const DeviceInfo* dev);
+
+// ------------------------------------------------------------ device side
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbarrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for the phase of `bar` with parity `parity` to complete. Gives up when
+// *abort becomes non-zero (another role gave up) or after limit_ns; on its own
+// expiry it raises *abort and the device error word. Returns true on success.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                  const DevErr& err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (abort != nullptr && *abort) return false;
+        if (globaltimer_ns() - t0 > err.limit_ns) {
+            if (abort != nullptr) *abort = 1;
+            atomicOr(err.word, kDevErrTimeout);
+            return false;
+        }
+    }
+}
+
+// TMA 2-D tiled load into shared memory, completion counted on `bar`.
+// Coordinates: x = inner (bytes for u8 tensors), y = row. No multicast.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
+                                            int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// ---- tcgen05 (one CTA per MMA: cta_group::1)
+__device__ __forceinline__ void tmem_alloc(uint32_t* smem_slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, E4M3 x E4M3 -> fp32.
+__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05.mma issued so far by this thread has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit TMEM columns -> 32 registers per thread.
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile stored the way
+// a 128-byte-swizzled TMA load leaves it: rows of 128 B, 8-row (1024 B)
+// swizzle atoms stacked along M/N. Fields (sm_100 UMMA descriptor): start
+// address >> 4 in bits 0-13, leading byte offset >> 4 in 16-29 (unused for
+// swizzled K-major, set to 1), stride byte offset >> 4 in 32-45 (1024 B
+// between 8-row groups), version 1 in bits 46-47, swizzle mode in 61-63
+// (2 = 128 B).
+__device__ __forceinline__ uint64_t umma_desc_kmajor_sw128(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
+// Instruction descriptor of kind::f8f6f4, E4M3 x E4M3 -> F32, both K-major.
+// Bits: D format 4-5 (1 = F32), A format 7-9 (0 = E4M3), B format 10-12,
+// A / B major 15 / 16 (0 = K), N >> 3 in 17-22, M >> 4 in 24-28.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3_f32(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace fp8dit

@@ -1,0 +1,203 @@
+/*
+ * fp8dit — FP8 linear layer of a diffusion / video DiT on B200 (sm_100a).
+ *
+ * The path (from "从 BF16 到 FP8：HunyuanVideo1.5推理优化复盘", section 三.1):
+ *
+ *     BF16 activation -> dynamic per-token FP8 quant -> FP8 GEMM
+ *                     -> scale / bias / output dtype
+ *
+ * with weights quantised per output channel ahead of time (section 二),
+ * one quantised activation shared by the Q, K and V projections (section
+ * 三.4), an entry that takes an already-quantised (fp8, scale) activation
+ * (sections 三.3 and 三.5), and the backend / tile choice bound once when a
+ * layer is created (section 三.3). The companion step converts whole weight
+ * tensors to float8_e4m3fn or float8_e5m2 with one scale each ("Quantize
+ * Model to FP8 Format", inputs model_state_dict and fp8_format).
+ *
+ * Quantisation recipe ("ComfyUI自定义节点开发适配Stable Diffusion 3.5 FP8技术要点",
+ * section "FP8：不只是精度减半", steps 1-4), read for FP8:
+ *     amax = max |x|                      (over a row, a channel or a tensor)
+ *     S    = fp32(amax) / fmax            IEEE fp32 division; S = 1 if amax == 0
+ *     q    = RNEsat(fp32(x) / S)          IEEE fp32 division, then round to the
+ *                                         nearest FP8 code (ties to even
+ *                                         mantissa), |.| > fmax clamps to fmax
+ *     x   ~= decode(q) * S                (the stored scale is S)
+ * fmax = 448 for E4M3FN, 57344 for E5M2.
+ *
+ * Conventions for every entry point
+ *  - bf16 tensors are passed as uint16_t bit patterns, FP8 tensors as uint8_t
+ *    codes (OCP E4M3FN / E5M2), scales as fp32. All tensors are row-major;
+ *    "K-major" means the reduction index is the contiguous one.
+ *  - Every tensor pointer is a DEVICE pointer on the current device unless a
+ *    parameter says "host". The caller owns all memory: inputs, outputs,
+ *    scratch and workspace. The library owns only linear handles.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and enqueue work only after every argument has been validated.
+ *    An argument error returns a status and enqueues nothing. There is no
+ *    fallback path: a shape the kernels cannot take is an error.
+ *  - Device-side bounded waits that expire set a per-device error word;
+ *    fp8dit_device_error() reads and clears it.
+ *  - On any status other than FP8DIT_OK, fp8dit_last_error_string() (per
+ *    thread) describes the failure.
+ */
+#ifndef FP8DIT_H
+#define FP8DIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8DIT_OK = 0,
+    FP8DIT_ERR_INVALID_ARG = 1,       /* null / misaligned pointer, negative size, bad format */
+    FP8DIT_ERR_UNSUPPORTED_SHAPE = 2, /* K % 16 != 0, N % 8 != 0, size beyond the kernels' range */
+    FP8DIT_ERR_EMPTY = 3,             /* per-tensor conversion with nothing to convert */
+    FP8DIT_ERR_CUDA = 4,              /* a CUDA runtime / driver call failed */
+    FP8DIT_ERR_TIMEOUT = 5            /* a bounded device wait expired */
+} fp8dit_status;
+
+typedef enum { FP8DIT_E4M3FN = 0, FP8DIT_E5M2 = 1 } fp8dit_format;
+
+/* Same type as cudaStream_t; the header does not need the CUDA headers. */
+typedef struct CUstream_st* fp8dit_stream_t;
+
+/* Opaque handle of one FP8 linear layer (see fp8_linear_create). */
+typedef struct fp8dit_linear_s* fp8dit_linear;
+
+/*
+ * Per-token (rowwise) quantisation of a bf16 activation.
+ * ("从 BF16 到 FP8", section 三.1: dynamic per-token FP8 quant; recipe above.)
+ *   x     [M, K] bf16, row stride ldx elements (ldx >= K, ldx % 8 == 0), 16-byte aligned.
+ *   q     [M, K] FP8 codes of format fmt, row stride ldq bytes (ldq >= K, ldq % 16 == 0),
+ *         16-byte aligned.
+ *   scale [M] fp32: S of each row.
+ * Requires K % 16 == 0 and K > 0, M >= 0 (M == 0 is a no-op). Any K that is a
+ * multiple of 16 is accepted. Inputs must be finite.
+ */
+fp8dit_status fp8_quantize_rowwise(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                   fp8dit_format fmt, uint8_t* q, int64_t ldq, float* scale,
+                                   fp8dit_stream_t stream);
+
+/*
+ * Per-output-channel quantisation of a bf16 weight W [N, K] (K contiguous):
+ * the rowwise recipe applied to each of the N rows, producing the K-major
+ * FP8 weight the GEMM consumes with no transpose ("从 BF16 到 FP8", section
+ * 二: parameters quantised per channel ahead of time; section 三.1: B must
+ * stay column-major, never transposed and made contiguous).
+ *   w [N, K] bf16 contiguous; qw [N, K] codes contiguous; sw [N] fp32.
+ * Requires N > 0, K > 0, K % 16 == 0.
+ */
+fp8dit_status fp8_quantize_weight_per_channel(const uint16_t* w, int64_t N, int64_t K,
+                                              fp8dit_format fmt, uint8_t* qw, float* sw,
+                                              fp8dit_stream_t stream);
+
+/* One tensor of a per-tensor conversion. Pointers are device pointers. */
+typedef struct {
+    const uint16_t* src; /* numel bf16 values, contiguous, 16-byte aligned */
+    int64_t numel;       /* >= 0; numel % 8 == 0 */
+    uint8_t* dst;        /* numel FP8 codes, 16-byte aligned */
+    float* scale;        /* one fp32: S of the tensor (left untouched when numel == 0) */
+} fp8dit_tensor_desc;
+
+/* Bytes of device workspace fp8_quantize_weight_per_tensor needs for n tensors. */
+size_t fp8_quantize_weight_per_tensor_workspace_size(int32_t n_tensors);
+
+/*
+ * Per-tensor conversion of a weight set (a state-dict's tensors) to FP8 with
+ * one amax scale per tensor ("Quantize Model to FP8 Format": model_state_dict
+ * in, quantised state-dict out in float8_e4m3fn or float8_e5m2).
+ *   tensors   HOST array of n_tensors descriptors; it may be freed on return.
+ *   workspace DEVICE scratch of at least
+ *             fp8_quantize_weight_per_tensor_workspace_size(n_tensors) bytes,
+ *             16-byte aligned; its contents on entry do not matter. It must not
+ *             be used by another call that runs at the same time on the GPU.
+ * Errors: FP8DIT_ERR_EMPTY when n_tensors == 0 or every numel is 0 (the page's
+ * "Invalid input." and "No tensor converted to <fp8_format>." outcomes).
+ */
+fp8dit_status fp8_quantize_weight_per_tensor(const fp8dit_tensor_desc* tensors, int32_t n_tensors,
+                                             fp8dit_format fmt, void* workspace, size_t ws_bytes,
+                                             fp8dit_stream_t stream);
+
+/*
+ * Create an FP8 linear layer y = (A W^T) * sa * sw + bias with E4M3FN
+ * operands, fp32 accumulation and bf16 output. The tile plan for every
+ * M-bucket and the weight's TMA descriptors are built here, once
+ * ("从 BF16 到 FP8", section 三.3: backend chosen from weight shape, device
+ * and bias contract at construction, forward does no such checks).
+ *   qw   [N, K] E4M3FN codes, K contiguous (from fp8_quantize_weight_per_channel).
+ *   sw   [N] fp32 per-channel scales.
+ *   bias [N] bf16, or NULL for no bias.
+ * The handle BORROWS qw, sw and bias: they must stay valid and unchanged
+ * until fp8_linear_destroy. device is the CUDA device that holds them.
+ * Requires N % 8 == 0, K % 16 == 0, qw 16-byte aligned.
+ */
+fp8dit_status fp8_linear_create(int64_t N, int64_t K, const uint8_t* qw, const float* sw,
+                                const uint16_t* bias, int device, fp8dit_linear* out);
+
+fp8dit_status fp8_linear_destroy(fp8dit_linear h);
+
+/*
+ * Forward of one FP8 linear layer ("从 BF16 到 FP8", sections 三.1, 三.3, 三.5):
+ *  - ordinary tensor: a_bf16 != NULL. A [M, K] bf16 (contiguous) is quantised
+ *    per token into qa_scratch [M, K] and sa_scratch [M] (both caller-owned,
+ *    written by this call), then multiplied. qa and sa must be NULL.
+ *  - FP8 tensor: a_bf16 == NULL. qa [M, K] E4M3FN codes (contiguous) and
+ *    sa [M] fp32 per-token scales are used as given; the scratch arguments
+ *    are ignored.
+ *   y [M, N] bf16 contiguous, 16-byte aligned:
+ *     y[m, n] = bf16_rne((sum_k dec(qa[m,k]) dec(qw[n,k])) * sa[m] * sw[n] + bias[n])
+ * M == 0 is a no-op. Must run on the handle's device.
+ */
+fp8dit_status fp8_scaled_linear(fp8dit_linear h, int64_t M, const uint16_t* a_bf16,
+                                const uint8_t* qa, const float* sa, uint8_t* qa_scratch,
+                                float* sa_scratch, uint16_t* y, fp8dit_stream_t stream);
+
+/*
+ * n linear layers that read the same activation ("从 BF16 到 FP8", section
+ * 三.4: quantise hidden_states once and feed the separate Q, K and V
+ * projections). A [M, K] bf16 is quantised once into qa_scratch / sa_scratch,
+ * then all n products run in one grouped launch.
+ *   hs  HOST array of n handles (1 <= n <= 4), all with the same K and device.
+ *   ys  HOST array of n device pointers, ys[i] is [M, N_i] bf16.
+ * Results are bitwise identical to n fp8_scaled_linear calls.
+ */
+fp8dit_status fp8_scaled_linear_multi(const fp8dit_linear* hs, int32_t n, int64_t M,
+                                      const uint16_t* a_bf16, uint8_t* qa_scratch,
+                                      float* sa_scratch, uint16_t* const* ys,
+                                      fp8dit_stream_t stream);
+
+/*
+ * Tile plan that fp8_scaled_linear / _multi use for this handle at this M
+ * (n_problems = 1 for a single layer): block_m x block_n output tiles,
+ * `ctas` thread blocks. For reports and tests.
+ */
+fp8dit_status fp8_linear_plan(fp8dit_linear h, int64_t M, int32_t n_problems, int32_t* block_m,
+                              int32_t* block_n, int32_t* ctas);
+
+/*
+ * Synchronise `stream`, then read and clear the current device's error word.
+ * Returns FP8DIT_ERR_TIMEOUT if a bounded device wait expired since the last
+ * read, FP8DIT_ERR_CUDA if the synchronisation failed, else FP8DIT_OK.
+ */
+fp8dit_status fp8dit_device_error(fp8dit_stream_t stream);
+
+/*
+ * Launch one block whose single thread waits, with the library's bounded
+ * wait, on an mbarrier that nothing arrives at, for at most limit_ns
+ * nanoseconds (1e3 .. 1e10). The wait expires and sets the error word, so
+ * the next fp8dit_device_error() reports FP8DIT_ERR_TIMEOUT. Exercises the
+ * failure path without faulting the GPU.
+ */
+fp8dit_status fp8dit_selftest_expired_wait(int64_t limit_ns, fp8dit_stream_t stream);
+
+/* Description of the last failure on this thread ("" if none). */
+const char* fp8dit_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8DIT_H */

@@ -26,3 +26,37 @@ def read_golden(name: str):
             if line:
                 rows.append(line.split())
     return rows
+
+
+# ------------------------------------------------------------ GPU helpers
+def to_device_bf16(a, device="cuda"):
+    """numpy uint16 bf16 patterns -> torch bf16 tensor on the device (same bytes)."""
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def to_host_u16(t):
+    import numpy as np
+    import torch
+    return t.detach().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_tensor_to_f64(t):
+    import numpy as np
+    return ((to_host_u16(t).astype(np.uint32) << 16).view(np.float32)).astype(np.float64)
+
+
+def canary_buffer(nbytes, margin=4096, device="cuda"):
+    """A uint8 buffer filled with 0xCD and a view of nbytes in its middle
+    (16-byte aligned); check_canary() verifies the margins are untouched."""
+    import torch
+    buf = torch.full((nbytes + 2 * margin,), 0xCD, dtype=torch.uint8, device=device)
+    return buf, buf[margin: margin + nbytes]
+
+
+def check_canary(buf, nbytes, margin=4096):
+    import torch
+    head = buf[:margin]
+    tail = buf[margin + nbytes:]
+    assert bool(torch.all(head == 0xCD)) and bool(torch.all(tail == 0xCD)), "write outside the output buffer"
