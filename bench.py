@@ -1,0 +1,503 @@
+"""Benchmark of the FP8 DiT linear hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp8dit|reference] [--no-extras]
+
+One step = the two FFN linears of a DiT block at the pages' shapes
+("从 BF16 到 FP8：HunyuanVideo1.5推理优化复盘", section 三.2), each the full
+path from a bf16 activation (section 三.1):
+  FFN-up   A [4096, 2048] -> per-token E4M3 quant -> GEMM vs W [8192, 2048] -> scale/bias/bf16
+  FFN-down A [4096, 8192] -> per-token E4M3 quant -> GEMM vs W [2048, 8192] -> scale/bias/bf16
+Inputs are synthetic (seeded, see synth/), resident in HBM before timing;
+three rotating input/output sets (~0.7 GB) keep every step's operands out of
+L2 (126 MB). Timing: CUDA events on the launching stream, W warm-up steps,
+K timed steps between a barrier + synchronize on both sides, max over ranks.
+
+`value` = FP8 linear TFLOP/s (2MNK per linear, quantisation time included).
+Also reported: the quantiser's HBM GB/s, per-kernel times, a roofline of the
+dominant kernel (the GEMM), NVML clocks during the timed region, an
+end-to-end figure through the public API with host buffers, and (N=1) the
+CPU oracle timed on the host as a baseline. `--impl reference` times the CPU
+oracle alone on bounded samples of the same workload.
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload with no
+data-path collective (weak scaling); only the timing uses the process group.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "fused FP8 linear TFLOP/s (% FP8 peak) at FFN shapes; quantizer GB/s (% HBM)"
+WORKLOAD = "FFN-up 4096x8192x2048 + FFN-down 4096x2048x8192 FP8 linear from bf16 activations"
+FFN = (("up", 4096, 8192, 2048), ("down", 4096, 2048, 8192))
+FLOPS_PER_STEP = sum(2.0 * M * N * K for _, M, N, K in FFN)
+# Quantiser algorithmic bytes: bf16 read + FP8 write + fp32 scale per row.
+QBYTES = {name: 2 * M * K + M * K + 4 * M for name, M, N, K in FFN}
+FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def config_dict(n_gpus: int) -> dict:
+    return {"workload": WORKLOAD, "a_dist": "up: N(0,1)+0.5% x30; down: GELU(N(0,1))",
+            "w_dist": "up N(0,0.02), down N(0,0.015), per-channel E4M3FN", "seed": 0,
+            "l2": "3 rotating input/output sets (~0.7 GB > L2)", "parallelism": f"replicas x{n_gpus}"}
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """NVML sampling of SM clock and throttle reasons during the timed region."""
+    REASONS = {
+        "hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80, "sync_boost": 0x10,
+    }
+
+    def __init__(self, torch_device, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reason_bits = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            import torch
+            props = torch.cuda.get_device_properties(torch_device)
+            try:  # NVML enumerates physical GPUs; match the CUDA device by UUID
+                self._h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # reported, not fatal
+            self._nvml = None
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reason_bits |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self) -> dict:
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = [k for k, bit in self.REASONS.items() if self.reason_bits & bit]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for rel in ("dit_rowwise_amax_b200/csrc/gemm_sm100.cu", "dit_rowwise_amax_b200/csrc/fp8dit_internal.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d.get(kernel)
+        if e and e.get("source_digest") == kernel_source_digest():
+            return e.get("bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------ CPU oracle leg
+def oracle_sample_step(data, rows: int):
+    """The oracle on the first `rows` rows of both FFN linears: per-token
+    quantisation of A, per-channel of W (prepared once), exact GEMM + epilogue."""
+    import oracle
+    flops = 0.0
+    for name, M, N, K in FFN:
+        d = data[name]
+        qa, sa = oracle.quantize_rows(d["A"][:rows], oracle.E4M3FN)
+        oracle.linear(qa, sa, d["qw"], d["sw"], d["bias"])
+        flops += 2.0 * rows * N * K
+    return flops
+
+
+def oracle_data():
+    import oracle
+    import synth
+    data = {"up": synth.ffn_up(), "down": synth.ffn_down()}
+    for d in data.values():
+        d["qw"], d["sw"] = oracle.quantize_rows(d["W"], oracle.E4M3FN)
+    return data
+
+
+def calibrate_rows(data, target_s: float) -> int:
+    import oracle
+    probe = max(2, oracle.num_threads())  # the oracle parallelises over rows
+    t0 = time.perf_counter()
+    oracle_sample_step(data, probe)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    return int(max(probe, min(4096, probe * target_s / dt)))
+
+
+def cpu_baseline(target_s: float = 12.0) -> dict:
+    import oracle
+    data = oracle_data()
+    rows = calibrate_rows(data, target_s)
+    t0 = time.perf_counter()
+    flops = oracle_sample_step(data, rows)
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {rows} rows of both FFN linears (quantise + exact GEMM + epilogue), {dt:.1f} s",
+            "cpu": cpu_model()}
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle as the reference arm: each step one bounded sample."""
+    if rank != 0:
+        return
+    import oracle
+    data = oracle_data()
+    rows = calibrate_rows(data, 1.5)
+    for _ in range(args.warmup):
+        oracle_sample_step(data, rows)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += oracle_sample_step(data, rows)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = f"first {rows} rows of both FFN linears per step (quantise + exact GEMM + epilogue)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64 exact / f64",
+        "data": "synthetic", "config": config_dict(world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample, "cpu": cpu_model()},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU leg
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("fp8dit", "reference"), default="fp8dit")
+    ap.add_argument("--no-extras", action="store_true", help="skip the attention / state-dict / bf16 extras")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import dit_rowwise_amax_b200 as fp8
+    import synth
+
+    fp8.load_library()  # fails loudly if the CUDA library is missing
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    host = {"up": synth.ffn_up(), "down": synth.ffn_down()}
+    layers = {name: fp8.FP8Linear.from_weight(up(host[name]["W"]), up(host[name]["bias"])) for name, *_ in FFN}
+    R = 3
+    sets = []
+    for _ in range(R):
+        s = {}
+        for name, M, N, K in FFN:
+            s[name] = {"A": up(host[name]["A"]),
+                       "qa": torch.empty((M, K), dtype=torch.uint8, device=dev),
+                       "sa": torch.empty((M,), dtype=torch.float32, device=dev),
+                       "y": torch.empty((M, N), dtype=torch.bfloat16, device=dev)}
+        sets.append(s)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, evs=None):
+        s = sets[i % R]
+        for j, (name, M, N, K) in enumerate(FFN):
+            b = s[name]
+            if evs is not None:
+                evs[2 * j].record(stream)
+            fp8.quantize_rowwise(b["A"], fp8.E4M3FN, q=b["qa"], scale=b["sa"])
+            if evs is not None:
+                evs[2 * j + 1].record(stream)
+            layers[name].forward_fp8(b["qa"], b["sa"], y=b["y"])
+        if evs is not None:
+            evs[4].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if fp8.device_error(dev) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    if fp8.device_error(dev) != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # Per-kernel averages over the timed region.
+    k_ms = {"quantize_up": [], "gemm_up": [], "quantize_down": [], "gemm_down": []}
+    for e in evs:
+        k_ms["quantize_up"].append(e[0].elapsed_time(e[1]))
+        k_ms["gemm_up"].append(e[1].elapsed_time(e[2]))
+        k_ms["quantize_down"].append(e[2].elapsed_time(e[3]))
+        k_ms["gemm_down"].append(e[3].elapsed_time(e[4]))
+    k_avg = {k: sum(v) / len(v) for k, v in k_ms.items()}
+
+    value = world * FLOPS_PER_STEP * args.steps / (elapsed_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    region_s = elapsed_ms * 1e-3
+    sustained = region_s > 2.0
+    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    fp8_peak = bf16_peak * FP8_OVER_BF16
+    hbm_peak = peaks["hbm_gbs"]
+
+    gemm_us = (k_avg["gemm_up"] + k_avg["gemm_down"]) / 2 * 1e3
+    gemm_flops = 2.0 * 4096 * 8192 * 2048
+    gemm_tflops = gemm_flops / (gemm_us * 1e-6) / 1e12
+    traffic = profiled_traffic("gemm_e4m3_kernel")
+    roofline = {"bound": "tensor", "kernel": "gemm_e4m3_kernel (FFN-up and FFN-down, mean)",
+                "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
+                "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x {FP8_OVER_BF16:g} "
+                               f"(nominal FP8/BF16 ratio)"}
+    q_gbs = {n: QBYTES[n] / (k_avg[f"quantize_{n}"] * 1e-3) / 1e9 for n in ("up", "down")}
+    q_all = (QBYTES["up"] + QBYTES["down"]) / ((k_avg["quantize_up"] + k_avg["quantize_down"]) * 1e-3) / 1e9
+    quantizer = {"value": q_all, "unit": "GB/s", "frac_of_hbm": q_all / hbm_peak, "peak": hbm_peak,
+                 "ffn_up_gbs": q_gbs["up"], "ffn_down_gbs": q_gbs["down"],
+                 "bytes_per_step": QBYTES["up"] + QBYTES["down"]}
+
+    # End to end through the public API with pinned host buffers.
+    e2e = measure_e2e(fp8, torch, layers, host, dev, args, world)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (bf16 in/out, fp32 accumulate)",
+        "data": "synthetic", "config": config_dict(world),
+        "frac_of_fp8_peak": value / (fp8_peak * world),
+        "roofline": roofline, "quantizer": quantizer,
+        "kernels_us": {k: v * 1e3 for k, v in k_avg.items()},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk, "e2e": e2e,
+    }
+    if world == 1 and rank == 0 and not args.no_extras:
+        line["extras"] = measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_e2e(fp8, torch, layers, host, dev, args, world):
+    """Same metric through FP8Linear.forward with host buffers: every step copies
+    both activations host->device (pinned) and both outputs device->host."""
+    pinned = {}
+    for name, M, N, K in FFN:
+        a = torch.from_numpy(np.ascontiguousarray(host[name]["A"]).view(np.int16)).view(torch.bfloat16)
+        pinned[name] = {"A": a.pin_memory(), "y": torch.empty((M, N), dtype=torch.bfloat16).pin_memory(),
+                        "Ad": torch.empty((M, K), dtype=torch.bfloat16, device=dev),
+                        "yd": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+                        "qa": torch.empty((M, K), dtype=torch.uint8, device=dev),
+                        "sa": torch.empty((M,), dtype=torch.float32, device=dev)}
+    h2d = sum(2 * M * K for _, M, N, K in FFN)
+    d2h = sum(2 * M * N for _, M, N, K in FFN)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for name, *_ in FFN:
+            p = pinned[name]
+            p["Ad"].copy_(p["A"], non_blocking=True)
+            layers[name].forward(p["Ad"], y=p["yd"], qa_scratch=p["qa"], sa_scratch=p["sa"])
+            p["y"].copy_(p["yd"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 50))
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * FLOPS_PER_STEP * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "api": "FP8Linear.forward (fp8_scaled_linear) + pinned host copies"}
+
+
+def time_region(torch, fn, iters, dev, warm=3):
+    stream = torch.cuda.current_stream(dev)
+    for i in range(warm):
+        fn(i)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(iters):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
+    out = {}
+    # Attention projections: hidden [32760, 2048] quantised once, Q / K / V in one grouped launch.
+    att = synth.attention()
+    layers = [fp8.FP8Linear.from_weight(up(att[f"W_{p}"]), up(att[f"bias_{p}"])) for p in "qkv"]
+    for name in ("hidden", "encoder"):
+        A = [up(att[name]) for _ in range(2)]
+        M = att[name].shape[0]
+        qa = torch.empty((M, 2048), dtype=torch.uint8, device=dev)
+        sa = torch.empty((M,), dtype=torch.float32, device=dev)
+        ys = [[torch.empty((M, 2048), dtype=torch.bfloat16, device=dev) for _ in range(3)] for _ in range(2)]
+        ms = time_region(torch, lambda i: fp8.scaled_linear_multi(layers, A[i % 2], ys=ys[i % 2], qa_scratch=qa,
+                                                                  sa_scratch=sa), 50, dev)
+        flops = 3 * 2.0 * M * 2048 * 2048
+        out[f"attention_qkv_{name}"] = {"M": M, "us": ms * 1e3, "tflops": flops / (ms * 1e-3) / 1e12,
+                                        "frac_of_fp8_peak": flops / (ms * 1e-3) / 1e12 / fp8_peak}
+        if name == "hidden":
+            qms = time_region(torch, lambda i: fp8.quantize_rowwise(A[i % 2], q=qa, scale=sa), 50, dev)
+            qb = 3 * M * 2048 + 4 * M
+            out["quantizer_hidden"] = {"us": qms * 1e3, "gbs": qb / (qms * 1e-3) / 1e9,
+                                       "frac_of_hbm": qb / (qms * 1e-3) / 1e9 / hbm_peak}
+    # GEMM only (pre-quantised activations) at the FFN shapes.
+    for name, M, N, K in FFN:
+        d = synth.ffn_up() if name == "up" else synth.ffn_down()
+        layer = fp8.FP8Linear.from_weight(up(d["W"]), up(d["bias"]))
+        qs = [fp8.quantize_rowwise(up(d["A"])) for _ in range(3)]
+        ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        ms = time_region(torch, lambda i: layer.forward_fp8(qs[i % 3][0], qs[i % 3][1], y=ys[i % 3]), 100, dev)
+        tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out[f"gemm_only_ffn_{name}"] = {"us": ms * 1e3, "tflops": tf, "frac_of_fp8_peak": tf / fp8_peak,
+                                        "plan": list(layer.plan(M))}
+        # BF16 context: the same shape through torch.matmul (cuBLAS), bench script only.
+        a16 = up(d["A"])
+        w16 = up(d["W"])
+        bms = time_region(torch, lambda i: torch.matmul(a16, w16.t()), 50, dev)
+        btf = 2.0 * M * N * K / (bms * 1e-3) / 1e12
+        out[f"bf16_torch_matmul_ffn_{name}"] = {"us": bms * 1e3, "tflops": btf}
+    # State-dict conversion: 192 tensors, 1.61e9 elements, both formats.
+    layout = synth.state_dict_layout()
+    tensors = []
+    for n, s in layout:
+        tensors.append(up(synth.state_dict_tensor(n, s)))
+    outs = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in tensors]
+    scales = torch.empty((len(tensors),), dtype=torch.float32, device=dev)
+    numel = sum(t.numel() for t in tensors)
+    alg_bytes = 3 * numel + 4 * len(tensors)
+    for fmt, fname in ((fp8.E4M3FN, "e4m3fn"), (fp8.E5M2, "e5m2")):
+        ms = time_region(torch, lambda i: fp8.quantize_per_tensor(tensors, fmt, outs=outs, scales=scales), 5, dev,
+                         warm=2)
+        out[f"state_dict_{fname}"] = {"tensors": len(tensors), "elements": numel, "us": ms * 1e3,
+                                      "gbs": alg_bytes / (ms * 1e-3) / 1e9,
+                                      "frac_of_hbm": alg_bytes / (ms * 1e-3) / 1e9 / hbm_peak}
+    return out
+
+
+if __name__ == "__main__":
+    main()

@@ -106,8 +106,9 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-fp8dit_status encode_tma_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+fp8dit_status encode_tma_2d(CUtensorMap* map, int elem_bytes, const void* base, uint64_t inner, uint64_t outer,
+                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                            CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) {
         set_error("cuTensorMapEncodeTiled is not available from the driver");
@@ -117,9 +118,9 @@ fp8dit_status encode_tma_2d_u8(CUtensorMap* map, const void* base, uint64_t inne
     const cuuint64_t strides[1] = {row_stride_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estride[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+    CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         set_error("cuTensorMapEncodeTiled failed (CUresult %d) for %llu x %llu", (int)r, (unsigned long long)outer,
                   (unsigned long long)inner);
@@ -161,31 +162,43 @@ struct fp8dit_linear_s {
     CUtensorMap tmB[kNumCfgs];  // weight descriptors, one per tile configuration
 };
 
-// Tile plan: 128 x 256 tiles unless they leave more than half the SMs idle,
-// then 128 x 128. Depends only on (M, N, n_problems, SM count).
+static int64_t tiles_for(const fp8dit_linear_s* h, int64_t M, int n_problems, int cfg) {
+    const int64_t bm = gemm_block_m(cfg), bn = gemm_block_n(cfg);
+    return ((M + bm - 1) / bm) * ((h->N + bn - 1) / bn) * n_problems;
+}
+
+// Tile plan, a function of (M, N, n_problems, SM count) only:
+//  - 256 x 256 tiles on CTA pairs when M fills a pair tile and the tiles keep
+//    at least half of the pairs busy;
+//  - else 128 x 256 tiles on single CTAs when they keep half the SMs busy;
+//  - else 128 x 128 tiles (small M: more CTAs, shorter latency).
 static int choose_cfg(const fp8dit_linear_s* h, int64_t M, int n_problems) {
-    const int64_t tm = (M + kGemmBlockM - 1) / kGemmBlockM;
-    const int64_t tiles256 = tm * ((h->N + 255) / 256) * n_problems;
-    return tiles256 * 2 >= h->num_sms ? kCfg128x256 : kCfg128x128;
+    const int pairs = h->num_sms / 2;
+    if (M >= 256 && tiles_for(h, M, n_problems, kCfgPair256) * 2 >= pairs) return kCfgPair256;
+    if (tiles_for(h, M, n_problems, kCfg128x256) * 2 >= h->num_sms) return kCfg128x256;
+    return kCfg128x128;
 }
 
 static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, const uint8_t* qa, const float* sa,
                               uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev) {
     const int cfg = choose_cfg(hs[0], M, n);
+    const int bm = gemm_block_m(cfg);
     const int bn = gemm_block_n(cfg);
     GemmArgs args;
     memset(&args, 0, sizeof(args));
-    fp8dit_status st = encode_tma_2d_u8(&args.tmA, qa, (uint64_t)hs[0]->K, (uint64_t)M, (uint64_t)hs[0]->K,
-                                        kGemmBlockK, kGemmBlockM, true);
+    fp8dit_status st = encode_tma_2d(&args.tmA, 1, qa, (uint64_t)hs[0]->K, (uint64_t)M, (uint64_t)hs[0]->K,
+                                     kGemmBlockK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FP8DIT_OK) return st;
-    const int tiles_m = (int)((M + kGemmBlockM - 1) / kGemmBlockM);
+    const int tiles_m = (int)((M + bm - 1) / bm);
     int tiles = 0;
     for (int g = 0; g < n; ++g) {
         args.tmB[g] = hs[g]->tmB[cfg];
+        st = encode_tma_2d(&args.tmY[g], 2, ys[g], (uint64_t)hs[g]->N, (uint64_t)M, (uint64_t)hs[g]->N * 2,
+                           kGemmStoreBox, kGemmStoreBox, CU_TENSOR_MAP_SWIZZLE_64B);
+        if (st != FP8DIT_OK) return st;
         GemmProblem& p = args.prob[g];
         p.sw = hs[g]->sw;
         p.bias = hs[g]->bias;
-        p.y = ys[g];
         p.N = (int32_t)hs[g]->N;
         p.tiles_n = (int32_t)((hs[g]->N + bn - 1) / bn);
         p.tile_start = tiles;
@@ -199,7 +212,7 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
     args.num_tiles = tiles;
     args.num_kb = (int32_t)((hs[0]->K + kGemmBlockK - 1) / kGemmBlockK);
     args.err = dev_err(dev);
-    cudaError_t e = launch_gemm(cfg, args, gemm_ctas_for(cfg, tiles, dev), stream);
+    cudaError_t e = launch_gemm(cfg, args, gemm_units_for(cfg, tiles, dev), stream);
     if (e != cudaSuccess) return cuda_fail(e, "FP8 GEMM launch");
     return FP8DIT_OK;
 }
@@ -307,8 +320,8 @@ fp8dit_status fp8_linear_create(int64_t N, int64_t K, const uint8_t* qw, const f
         h->device = device;
         h->num_sms = dev->num_sms;
         for (int cfg = 0; cfg < kNumCfgs && st == FP8DIT_OK; ++cfg)
-            st = encode_tma_2d_u8(&h->tmB[cfg], qw, (uint64_t)K, (uint64_t)N, (uint64_t)K, kGemmBlockK,
-                                  (uint32_t)gemm_block_n(cfg), true);
+            st = encode_tma_2d(&h->tmB[cfg], 1, qw, (uint64_t)K, (uint64_t)N, (uint64_t)K, kGemmBlockK,
+                               (uint32_t)gemm_b_box_rows(cfg), CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (device != prev) cudaSetDevice(prev);
     if (st != FP8DIT_OK) {
@@ -398,11 +411,11 @@ fp8dit_status fp8_linear_plan(fp8dit_linear h, int64_t M, int32_t n_problems, in
     t_last_error[0] = 0;
     if (!h || M < 0 || n_problems < 1 || n_problems > kMaxGroups) return invalid("plan arguments");
     const int cfg = choose_cfg(h, M, n_problems);
-    const int bn = gemm_block_n(cfg);
-    const int64_t tiles = ((M + kGemmBlockM - 1) / kGemmBlockM) * ((h->N + bn - 1) / bn) * n_problems;
-    if (block_m) *block_m = kGemmBlockM;
-    if (block_n) *block_n = bn;
-    if (ctas) *ctas = (int32_t)(tiles < h->num_sms ? tiles : h->num_sms);
+    const int64_t tiles = tiles_for(h, M, n_problems, cfg);
+    const int64_t max_units = h->num_sms / gemm_cta_group(cfg);
+    if (block_m) *block_m = gemm_block_m(cfg);
+    if (block_n) *block_n = gemm_block_n(cfg);
+    if (ctas) *ctas = (int32_t)((tiles < max_units ? tiles : max_units) * gemm_cta_group(cfg));
     return FP8DIT_OK;
 }
 

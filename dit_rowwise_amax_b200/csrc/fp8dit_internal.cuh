@@ -38,10 +38,11 @@ const DeviceInfo* device_info();
 void set_error(const char* fmt, ...);
 fp8dit_status cuda_fail(cudaError_t e, const char* what);
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point.
-fp8dit_status encode_tma_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                               bool swizzle128);
+// cuTensorMapEncodeTiled through the runtime's driver entry point: a 2-D
+// row-major tensor of 1- or 2-byte elements (inner = contiguous extent).
+fp8dit_status encode_tma_2d(CUtensorMap* map, int elem_bytes, const void* base, uint64_t inner, uint64_t outer,
+                            uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                            CUtensorMapSwizzle swizzle);
 
 // Launchers (each validates nothing; the API layer has done it).
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int fmt,
@@ -66,15 +67,15 @@ constexpr int kMaxGroups = 4;
 struct GemmProblem {
     const float* sw;
     const uint16_t* bias;  // may be null
-    uint16_t* y;
     int32_t N;
     int32_t tiles_n;
     int32_t tile_start;  // first global tile index of this problem
 };
 
 struct alignas(64) GemmArgs {
-    CUtensorMap tmA;
-    CUtensorMap tmB[kMaxGroups];
+    CUtensorMap tmA;               // A codes [M, K], box 128 x 128 B, 128-byte swizzle
+    CUtensorMap tmB[kMaxGroups];   // W codes [N, K], box rows per configuration
+    CUtensorMap tmY[kMaxGroups];   // y bf16 [M, N], box 32 x 32, 64-byte swizzle (TMA store)
     GemmProblem prob[kMaxGroups];
     const float* sa;
     int32_t M, K, G;
@@ -86,16 +87,20 @@ struct alignas(64) GemmArgs {
 
 // Tile configurations the plan chooses from.
 enum GemmConfig : int32_t {
-    kCfg128x256 = 0,
-    kCfg128x128 = 1,
-    kNumCfgs = 2,
+    kCfgPair256 = 0,  // 256 x 256 tile on a 2-CTA pair (cta_group::2)
+    kCfg128x256 = 1,  // 128 x 256 tile on one CTA
+    kCfg128x128 = 2,  // 128 x 128 tile on one CTA
+    kNumCfgs = 3,
 };
+int gemm_block_m(int cfg);
 int gemm_block_n(int cfg);
-constexpr int kGemmBlockM = 128;
+int gemm_b_box_rows(int cfg);
+int gemm_cta_group(int cfg);
 constexpr int kGemmBlockK = 128;  // bytes = FP8 elements per k-block (one 128 B swizzle row)
+constexpr int kGemmStoreBox = 32;
 
-cudaError_t launch_gemm(int cfg, const GemmArgs& args, int ctas, cudaStream_t stream);
-int gemm_ctas_for(int cfg, int num_tiles, const DeviceInfo* dev);
+cudaError_t launch_gemm(int cfg, const GemmArgs& args, int units, cudaStream_t stream);
+int gemm_units_for(int cfg, int num_tiles, const DeviceInfo* dev);
 
 // ------------------------------------------------------------ device side
 #if defined(__CUDACC__)
@@ -173,6 +178,97 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// ---- clusters (2-CTA MMA pairs)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// TMA load for a 2-CTA MMA pair: data lands in this CTA's shared memory, the
+// byte count is signalled on `mbar_cluster_addr`, which may be the leader
+// CTA's barrier. No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t mbar_cluster_addr,
+                                                 int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(map), "r"(mbar_cluster_addr), "r"(x), "r"(y)
+        : "memory");
+}
+
+// TMA store of a shared-memory box to global memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+                 "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// Order this thread's generic-proxy shared-memory writes before later async-proxy (TMA) reads.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ---- tcgen05 with two CTAs per MMA (cta_group::2): issued by the pair's leader.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive once on `bar` in every CTA of `cta_mask` when this thread's prior pair MMAs complete.
+__device__ __forceinline__ void mma_commit_pair_multicast(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 
 // ---- tcgen05 (one CTA per MMA: cta_group::1)

@@ -8,18 +8,29 @@
 // A [M, K] and W [N, K] are both K-major (the "column-major B" of section 三.1,
 // fixed at weight preparation, so no transpose ever reaches this kernel).
 //
-// Structure (one CTA per SM, persistent over output tiles):
+// Structure (persistent over output tiles, one CTA per SM):
 //   warp 0      one thread issues TMA loads of A and W k-blocks (128 B wide,
 //               128-byte swizzle) into a STAGES-deep shared-memory ring;
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN,
-//               K=32 per instruction) into a TMEM accumulator and commits
-//               each ring slot back to the producer when its MMAs retire;
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, scale, bias, bf16,
-//               16-byte global stores; then hand the accumulator back.
-// Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap
-// the mainloop of tile i+1. All mbarrier waits are bounded (see
-// mbar_wait_bounded): on expiry the CTA raises the device error word, drains
-// its in-flight copies and MMAs, frees TMEM and returns.
+//   warp 1      allocates TMEM; one thread of the pair's leader CTA issues
+//               tcgen05.mma (K = 32 per instruction) into a TMEM accumulator
+//               and commits each ring slot back to the producers;
+//   warps 2..5  epilogue: stage the tile's sw / bias in shared memory,
+//               tcgen05.ld 32 accumulator columns at a time, scale, bias,
+//               bf16, write a 32 x 32 box into a 64-byte-swizzled staging
+//               buffer and TMA-store it (double-buffered per warp).
+// Two TMEM accumulators let the epilogue of tile i overlap the mainloop of
+// tile i+1.
+//
+// CG = 2 runs one MMA across a CTA pair (cta_group::2, a 2-CTA cluster): the
+// tile is 256 x BN, each CTA loads its 128 rows of A and BN/2 rows of W, the
+// leader issues the MMAs, and each CTA's TMEM receives its 128 output rows.
+// Per-SM shared-memory traffic per MMA is half that of a 1-CTA tile, which
+// lets a 6-deep ring of 32 KB stages cover the L2 latency. No TMA load
+// anywhere uses multicast.
+//
+// Every mbarrier wait is bounded (mbar_wait_bounded): on expiry the CTA
+// raises the device error word and its own and its peer's abort flags, lets
+// in-flight copies and MMAs land, frees TMEM and returns.
 #include <cuda_bf16.h>
 
 #include "fp8dit_internal.cuh"
@@ -27,21 +38,30 @@
 namespace fp8dit {
 namespace {
 
-template <int BN>
+template <int CG, int BN>
 struct Cfg {
-    static constexpr int BM = kGemmBlockM;
-    static constexpr int BK = kGemmBlockK;
-    static constexpr int STAGES = BN == 256 ? 4 : 6;
-    static constexpr int A_BYTES = BM * BK;
-    static constexpr int B_BYTES = BN * BK;
+    static constexpr int BM = 128 * CG;    // rows of one MMA tile
+    static constexpr int ROWS = 128;       // rows per CTA (TMEM lanes)
+    static constexpr int BK = kGemmBlockK;  // 128 FP8 = one 128-byte swizzle row
+    static constexpr int B_ROWS = BN / CG;  // W rows per CTA per stage
+    static constexpr int A_BYTES = ROWS * BK;
+    static constexpr int B_BYTES = B_ROWS * BK;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int ACC = 2;  // TMEM accumulator buffers
+    static constexpr int STAGES = (CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6);
+    static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
+    static constexpr int EPI_WARPS = 4;
+    static constexpr int BOX = 32;                   // epilogue store box: 32 rows x 32 columns
+    static constexpr int STG_BYTES = BOX * BOX * 2;  // 2 KB, 64-byte rows
+    static constexpr int STAGING_BYTES = EPI_WARPS * 2 * STG_BYTES;
+    static constexpr int SWB_FLOATS = 2 * BN;        // sw then bias as fp32, one copy per epilogue warp
+    static constexpr int SWB_BYTES = EPI_WARPS * SWB_FLOATS * 4;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
     static constexpr int THREADS = 192;
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
     static_assert((2 * STAGES + 2 * ACC + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 struct TileCoord {
@@ -62,14 +82,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int BN>
-__global__ void __launch_bounds__(Cfg<BN>::THREADS, 1) gemm_e4m3_kernel(const __grid_constant__ GemmArgs args) {
-    using C = Cfg<BN>;
+template <int CG, int BN>
+__global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(const __grid_constant__ GemmArgs args) {
+    using C = Cfg<CG, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+    uint8_t* sB = sA + C::STAGES * C::A_BYTES;
+    uint8_t* staging = sB + C::STAGES * C::B_BYTES;
+    float* swb = reinterpret_cast<float*>(staging + C::STAGING_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(swb) + C::SWB_BYTES);
     uint64_t* empty = full + C::STAGES;
     uint64_t* tfull = empty + C::STAGES;
     uint64_t* tempty = tfull + C::ACC;
@@ -79,6 +101,15 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1) gemm_e4m3_kernel(const __
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = (CG == 2) ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // MMA unit (pair or CTA)
+    const int units = (CG == 2) ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+
+    // Tell the other CTA of the pair to stop waiting (after our own wait expired).
+    auto abort_peer = [&]() {
+        if (CG == 2) st_shared_cluster_u32(mapa_shared(smem_u32((const void*)abort_flag), rank ^ 1u), 1u);
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -87,39 +118,58 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1) gemm_e4m3_kernel(const __
         }
         for (int a = 0; a < C::ACC; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+            mbar_init(&tempty[a], C::EPI_WARPS * CG);  // one arrival per epilogue warp of the pair
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&args.tmA);
-        for (int g = 0; g < args.G; ++g) tma_prefetch_desc(&args.tmB[g]);
+        for (int g = 0; g < args.G; ++g) {
+            tma_prefetch_desc(&args.tmB[g]);
+            tma_prefetch_desc(&args.tmY[g]);
+        }
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
+        if (CG == 2) {
+            tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync_all();  // peer barriers initialised before any remote signal
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    bool aborted = false;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
             int64_t armed = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
+            for (int t = unit; t < args.num_tiles && !aborted; t += units) {
                 const TileCoord tc = tile_coord(args, t);
+                const int a_row = tc.tm * C::BM + (int)rank * C::ROWS;
+                const int b_row = tc.tn * BN + (int)rank * C::B_ROWS;
                 for (int kb = 0; kb < args.num_kb; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.err)) {
-                        ok = false;
+                        aborted = true;
+                        abort_peer();
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-                    tma_load_2d(sA + stage * C::A_BYTES, &args.tmA, &full[stage], kb * C::BK, tc.tm * C::BM);
-                    tma_load_2d(sB + stage * C::B_BYTES, &args.tmB[tc.g], &full[stage], kb * C::BK, tc.tn * BN);
+                    if (CG == 2) {
+                        const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], CG * C::STAGE_BYTES);
+                        tma_load_2d_pair(sA + stage * C::A_BYTES, &args.tmA, bar, kb * C::BK, a_row);
+                        tma_load_2d_pair(sB + stage * C::B_BYTES, &args.tmB[tc.g], bar, kb * C::BK, b_row);
+                    } else {
+                        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+                        tma_load_2d(sA + stage * C::A_BYTES, &args.tmA, &full[stage], kb * C::BK, a_row);
+                        tma_load_2d(sB + stage * C::B_BYTES, &args.tmB[tc.g], &full[stage], kb * C::BK, b_row);
+                    }
                     ++armed;
                     if (++stage == C::STAGES) {
                         stage = 0;
@@ -127,77 +177,102 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1) gemm_e4m3_kernel(const __
                     }
                 }
             }
-            if (!ok) {
-                // Let every copy this thread started land before the CTA exits.
-                DevErr drain_err = args.err;
+            if (aborted && leader) {
+                // Let every copy signalled on this CTA's barriers land before exit.
                 for (int s = 0; s < C::STAGES; ++s) {
                     if (armed <= s) break;
                     const int64_t last = s + (int64_t)C::STAGES * ((armed - 1 - s) / C::STAGES);
-                    mbar_wait_bounded(&full[s], (uint32_t)((last / C::STAGES) & 1), nullptr, drain_err);
+                    mbar_wait_bounded(&full[s], (uint32_t)((last / C::STAGES) & 1), nullptr, args.err);
                 }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------ MMA issuer (pair leader)
+        if (lane == 0 && leader) {
             constexpr uint32_t idesc = umma_idesc_e4m3_f32(C::BM, BN);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < args.num_tiles && ok; t += gridDim.x) {
+            for (int t = unit; t < args.num_tiles && !aborted; t += units) {
                 if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, args.err)) {
-                    ok = false;
+                    aborted = true;
+                    abort_peer();
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 for (int kb = 0; kb < args.num_kb; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, args.err)) {
-                        ok = false;
+                        aborted = true;
+                        abort_peer();
                         break;
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
                     const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-                    for (int j = 0; j < C::BK / 32; ++j)
-                        mma_f8f6f4(d_tmem, umma_desc_kmajor_sw128(a0 + 32 * j), umma_desc_kmajor_sw128(b0 + 32 * j),
-                                   idesc, (kb | j) != 0);
-                    mma_commit(&empty[stage]);  // slot free once these MMAs have read it
+                    for (int j = 0; j < C::BK / 32; ++j) {
+                        const uint64_t ad = umma_desc_kmajor_sw128(a0 + 32 * j);
+                        const uint64_t bd = umma_desc_kmajor_sw128(b0 + 32 * j);
+                        if (CG == 2) mma_f8f6f4_pair(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                        else mma_f8f6f4(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                    }
+                    // The ring slot is free (in both CTAs) once these MMAs have read it.
+                    if (CG == 2) mma_commit_pair_multicast(&empty[stage], 0x3);
+                    else mma_commit(&empty[stage]);
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (!ok) break;
-                mma_commit(&tfull[acc]);  // accumulator ready for the epilogue
+                if (aborted) break;
+                if (CG == 2) mma_commit_pair_multicast(&tfull[acc], 0x3);
+                else mma_commit(&tfull[acc]);
                 if (++acc == C::ACC) {
                     acc = 0;
                     acc_phase ^= 1u;
                 }
             }
             // Every MMA this thread issued has completed once `drain` fires.
-            mma_commit(drain);
+            if (CG == 2) mma_commit_pair(drain);
+            else mma_commit(drain);
             mbar_wait_bounded(drain, 0, nullptr, args.err);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps
-        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32)
+        const int q = warp & 3;     // TMEM lane quarter this warp may access
+        const int ew = warp - 2;    // this warp's staging buffers and scale copy
+        uint8_t* stg = staging + ew * 2 * C::STG_BYTES;
+        float* sw_s = swb + ew * C::SWB_FLOATS;
+        float* b_s = sw_s + BN;
         uint32_t acc = 0, acc_phase = 0;
-        for (int t = blockIdx.x; t < args.num_tiles; t += gridDim.x) {
+        uint32_t stores = 0;
+        for (int t = unit; t < args.num_tiles; t += units) {
             const TileCoord tc = tile_coord(args, t);
+            const GemmProblem& P = args.prob[tc.g];
+            // Stage this tile's per-channel scales and bias (as fp32) in this
+            // warp's own copy: no cross-warp barrier, so a warp that stops early
+            // on an expired wait cannot stall the others.
+            for (int j = lane; j < BN; j += 32) {
+                const int n = tc.tn * BN + j;
+                const bool in = n < P.N;
+                sw_s[j] = in ? __ldg(P.sw + n) : 0.0f;
+                b_s[j] = (in && P.bias != nullptr) ? __uint_as_float((uint32_t)__ldg(P.bias + n) << 16) : 0.0f;
+            }
+            __syncwarp();
+            const int row0 = tc.tm * C::BM + (int)rank * C::ROWS + q * 32;  // first row of this warp's box
+            const int row = row0 + lane;
+            const float sa = row < args.M ? __ldg(args.sa + row) : 0.0f;
+
             // Every lane waits; the warp then agrees (and reconverges) before
             // the warp-collective TMEM loads.
             const bool ready = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, args.err);
-            if (!__all_sync(0xffffffffu, ready)) break;
+            if (!__all_sync(0xffffffffu, ready)) {
+                if (lane == 0) abort_peer();
+                break;
+            }
             tc_fence_after();
-            const GemmProblem& P = args.prob[tc.g];
-            const int row = tc.tm * C::BM + quarter * 32 + lane;
-            const bool row_ok = row < args.M;
-            const float sa = row_ok ? __ldg(args.sa + row) : 0.0f;
-            uint16_t* yrow = P.y + (int64_t)(row_ok ? row : 0) * P.N;
-            const uint32_t t_addr = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+            const uint32_t t_addr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 const int n0 = tc.tn * BN + c * 32;
@@ -205,80 +280,121 @@ __global__ void __launch_bounds__(Cfg<BN>::THREADS, 1) gemm_e4m3_kernel(const __
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_addr + c * 32, r);
                 tmem_wait_ld();
+                uint32_t packed[16];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int n = n0 + q * 8;
-                    if (n < P.N) {
-                        const float4 w0 = __ldg(reinterpret_cast<const float4*>(P.sw + n));
-                        const float4 w1 = __ldg(reinterpret_cast<const float4*>(P.sw + n + 4));
-                        uint4 bb = make_uint4(0, 0, 0, 0);
-                        if (P.bias != nullptr) bb = __ldg(reinterpret_cast<const uint4*>(P.bias + n));
-                        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                        const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-                        float o[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float b = __uint_as_float(e & 1 ? (bw[e >> 1] & 0xffff0000u) : (bw[e >> 1] << 16));
-                            o[e] = fmaf(__uint_as_float(r[q * 8 + e]) * sa, wv[e], b);
-                        }
-                        uint4 packed;
-                        packed.x = pack_bf16x2(o[0], o[1]);
-                        packed.y = pack_bf16x2(o[2], o[3]);
-                        packed.z = pack_bf16x2(o[4], o[5]);
-                        packed.w = pack_bf16x2(o[6], o[7]);
-                        if (row_ok) *reinterpret_cast<uint4*>(yrow + n) = packed;
-                    }
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(sw_s + c * 32 + j);
+                    const float4 b4 = *reinterpret_cast<const float4*>(b_s + c * 32 + j);
+                    const float o0 = fmaf(__uint_as_float(r[j + 0]) * sa, w4.x, b4.x);
+                    const float o1 = fmaf(__uint_as_float(r[j + 1]) * sa, w4.y, b4.y);
+                    const float o2 = fmaf(__uint_as_float(r[j + 2]) * sa, w4.z, b4.z);
+                    const float o3 = fmaf(__uint_as_float(r[j + 3]) * sa, w4.w, b4.w);
+                    packed[j / 2] = pack_bf16x2(o0, o1);
+                    packed[j / 2 + 1] = pack_bf16x2(o2, o3);
                 }
+                uint8_t* buf = stg + (stores & 1u) * C::STG_BYTES;
+                if (stores >= 2) {
+                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+                    __syncwarp();
+                }
+                // Row `lane` of a 32 x 32 bf16 box, 64-byte rows, 64-byte swizzle.
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int phys = k4 ^ ((lane >> 1) & 3);
+                    *reinterpret_cast<uint4*>(buf + lane * 64 + phys * 16) =
+                        make_uint4(packed[4 * k4], packed[4 * k4 + 1], packed[4 * k4 + 2], packed[4 * k4 + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && row0 < args.M) {
+                    tma_store_2d(&args.tmY[tc.g], buf, n0, row0);
+                    bulk_commit_group();
+                }
+                ++stores;
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if (lane == 0) {
+                if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+                else mbar_arrive(&tempty[acc]);
+            }
             if (++acc == C::ACC) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
         }
+        if (lane == 0) bulk_wait_group<0>();  // all output stores complete
+        __syncwarp();
     }
 
+    if (*abort_flag) {
+        // Give copies that this CTA cannot wait for (a pair's follower signals
+        // the leader's barriers) time to land before shared memory is released.
+        const unsigned long long t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 50000ull) {
+        }
+    }
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync_all();  // both CTAs done with TMEM and each other's barriers
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if (CG == 2) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 
-template <int BN>
-cudaError_t launch_bn(const GemmArgs& args, int ctas, cudaStream_t stream) {
-    using C = Cfg<BN>;
+template <int CG, int BN>
+cudaError_t launch_cfg(const GemmArgs& args, int units, cudaStream_t stream) {
+    using C = Cfg<CG, BN>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_done[dev]) {
-        e = cudaFuncSetAttribute(gemm_e4m3_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        e = cudaFuncSetAttribute(gemm_e4m3_kernel<CG, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    gemm_e4m3_kernel<BN><<<ctas, C::THREADS, C::SMEM_BYTES, stream>>>(args);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units * CG), 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gemm_e4m3_kernel<CG, BN>, args);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int gemm_block_n(int cfg) { return cfg == kCfg128x256 ? 256 : 128; }
+int gemm_block_m(int cfg) { return cfg == kCfgPair256 ? 256 : 128; }
+int gemm_block_n(int cfg) { return cfg == kCfg128x128 ? 128 : 256; }
+int gemm_b_box_rows(int cfg) { return cfg == kCfg128x256 ? 256 : 128; }
+int gemm_cta_group(int cfg) { return cfg == kCfgPair256 ? 2 : 1; }
 
-int gemm_ctas_for(int cfg, int num_tiles, const DeviceInfo* dev) {
-    (void)cfg;
-    return num_tiles < dev->num_sms ? num_tiles : dev->num_sms;
+// MMA units (CTA pairs or CTAs) to launch: one per tile, at most one per SM (pair).
+int gemm_units_for(int cfg, int num_tiles, const DeviceInfo* dev) {
+    const int max_units = dev->num_sms / gemm_cta_group(cfg);
+    return num_tiles < max_units ? num_tiles : max_units;
 }
 
-cudaError_t launch_gemm(int cfg, const GemmArgs& args, int ctas, cudaStream_t stream) {
+cudaError_t launch_gemm(int cfg, const GemmArgs& args, int units, cudaStream_t stream) {
     switch (cfg) {
+        case kCfgPair256:
+            return launch_cfg<2, 256>(args, units, stream);
         case kCfg128x256:
-            return launch_bn<256>(args, ctas, stream);
+            return launch_cfg<1, 256>(args, units, stream);
         case kCfg128x128:
-            return launch_bn<128>(args, ctas, stream);
+            return launch_cfg<1, 128>(args, units, stream);
         default:
             return cudaErrorInvalidValue;
     }

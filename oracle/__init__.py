@@ -61,6 +61,8 @@ def _load():
         lib.or_linear.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p]
         lib.or_linear_at.restype = None
         lib.or_linear_at.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _p, _i64, _p]
+        lib.or_num_threads.restype = ctypes.c_int
+        lib.or_num_threads.argtypes = []
         lib.or_dot_units.restype = None
         lib.or_dot_units.argtypes = [_p, _p, _i64, _i64, _i64, _p]
         _lib = lib
@@ -143,6 +145,11 @@ def dot_units(qa, qw) -> np.ndarray:
     out = np.empty((M, N), dtype=np.int64)
     _load().or_dot_units(qa.ctypes.data, qw.ctypes.data, M, N, K, out.ctypes.data)
     return out
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use."""
+    return int(_load().or_num_threads())
 
 
 def tolerance_ok(gpu: np.ndarray, ref: np.ndarray, rms_ref: float | None = None):

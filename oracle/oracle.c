@@ -35,6 +35,7 @@
  * division with subnormals; no flush-to-zero).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -211,3 +212,6 @@ void or_encode_many(int fmt, const float* v, int64_t n, uint8_t* out) {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) out[i] = or_encode(fmt, v[i]);
 }
+
+/* Threads the oracle's parallel loops use (for reports). */
+int or_num_threads(void) { return omp_get_max_threads(); }
