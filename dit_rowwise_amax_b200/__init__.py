@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "E4M3FN", "E5M2", "Fp8DitError", "FP8Linear", "library_path", "load_library",
     "quantize_rowwise", "quantize_weight_per_channel", "quantize_per_tensor", "convert_state_dict",
-    "scaled_linear_multi", "device_error", "selftest_expired_wait", "as_float8",
+    "scaled_linear_multi", "device_error", "selftest_expired_wait", "selftest_quotient", "as_float8",
 ]
 
 E4M3FN = 0
@@ -76,10 +76,12 @@ def load_library():
     L.fp8_linear_plan.argtypes = [p, i64, i32, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.fp8dit_device_error.argtypes = [p]
     L.fp8dit_selftest_expired_wait.argtypes = [i64, p]
+    L.fp8dit_selftest_quotient.argtypes = [p, p]
     L.fp8dit_last_error_string.restype = ctypes.c_char_p
     for name in ("fp8_quantize_rowwise", "fp8_quantize_weight_per_channel", "fp8_quantize_weight_per_tensor",
                  "fp8_linear_create", "fp8_linear_destroy", "fp8_scaled_linear", "fp8_scaled_linear_multi",
-                 "fp8_linear_plan", "fp8dit_device_error", "fp8dit_selftest_expired_wait"):
+                 "fp8_linear_plan", "fp8dit_device_error", "fp8dit_selftest_expired_wait",
+                 "fp8dit_selftest_quotient"):
         getattr(L, name).restype = st
     _lib = L
     return L
@@ -319,3 +321,13 @@ def selftest_expired_wait(limit_ns: int = 2_000_000, device: Optional[torch.devi
     """Launch the bounded-wait self test (a wait that must expire)."""
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
     _check(load_library().fp8dit_selftest_expired_wait(limit_ns, _stream(dev)))
+
+
+def selftest_quotient(device: Optional[torch.device] = None) -> Tuple[int, int]:
+    """Run the exhaustive quotient self test; returns the FP8 code mismatch
+    counts (E4M3FN, E5M2) against IEEE division (both must be 0)."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    out = torch.zeros(2, dtype=torch.int64, device=dev)
+    _check(load_library().fp8dit_selftest_quotient(out.data_ptr(), _stream(dev)))
+    vals = out.cpu().tolist()
+    return int(vals[0]), int(vals[1])

@@ -446,4 +446,13 @@ fp8dit_status fp8dit_selftest_expired_wait(int64_t limit_ns, fp8dit_stream_t str
     return e == cudaSuccess ? FP8DIT_OK : cuda_fail(e, "self-test launch");
 }
 
+fp8dit_status fp8dit_selftest_quotient(unsigned long long* mismatch, fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (!mismatch || (reinterpret_cast<uintptr_t>(mismatch) & 7u)) return invalid("mismatch must be 8-byte aligned");
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    cudaError_t e = launch_selftest_quotient(mismatch, (cudaStream_t)stream);
+    return e == cudaSuccess ? FP8DIT_OK : cuda_fail(e, "quotient self-test launch");
+}
+
 }  // extern "C"

@@ -60,6 +60,7 @@ cudaError_t launch_per_tensor(const fp8dit_tensor_desc* host_descs, int32_t n, i
                               cudaStream_t stream, const DeviceInfo* dev, DevErr err);
 
 cudaError_t launch_selftest_wait(cudaStream_t stream, DevErr err);
+cudaError_t launch_selftest_quotient(unsigned long long* mismatch, cudaStream_t stream);
 
 // Grouped GEMM: up to kMaxGroups products sharing the quantised A.
 constexpr int kMaxGroups = 4;

@@ -14,8 +14,9 @@
 //   warp 1      allocates TMEM; one thread of the pair's leader CTA issues
 //               tcgen05.mma (K = 32 per instruction) into a TMEM accumulator
 //               and commits each ring slot back to the producers;
-//   warps 2..5  epilogue: stage the tile's sw / bias in shared memory,
-//               tcgen05.ld 32 accumulator columns at a time, scale, bias,
+//   warps 2..5  epilogue: fetch the next tile's sw / bias / sa while this
+//               tile is processed, tcgen05.ld 32 accumulator columns at a
+//               time, scale, bias,
 //               bf16, write a 32 x 32 box into a 64-byte-swizzled staging
 //               buffer and TMA-store it (double-buffered per warp).
 // Two TMEM accumulators let the epilogue of tile i overlap the mainloop of
@@ -245,24 +246,65 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
         uint8_t* stg = staging + ew * 2 * C::STG_BYTES;
         float* sw_s = swb + ew * C::SWB_FLOATS;
         float* b_s = sw_s + BN;
-        uint32_t acc = 0, acc_phase = 0;
-        uint32_t stores = 0;
-        for (int t = unit; t < args.num_tiles; t += units) {
+        constexpr int SW_V4 = BN / 4 / 32;  // float4 of sw per lane
+        constexpr int B_V8 = (BN / 8 + 31) / 32;  // 8-wide bf16 bias vectors per lane (lanes >= BN/8 idle)
+
+        // Per-tile epilogue operands, fetched one tile ahead: the scales and
+        // bias of the tile's columns, and sa of this lane's row. All loads of
+        // a tile are independent, so one memory round trip covers them, and
+        // it overlaps the previous tile's processing.
+        struct Pre {
+            float4 sw[SW_V4];
+            uint4 b[B_V8];
+            float sa;
+        };
+        auto fetch = [&](int t, Pre& p) {
             const TileCoord tc = tile_coord(args, t);
             const GemmProblem& P = args.prob[tc.g];
-            // Stage this tile's per-channel scales and bias (as fp32) in this
-            // warp's own copy: no cross-warp barrier, so a warp that stops early
-            // on an expired wait cannot stall the others.
-            for (int j = lane; j < BN; j += 32) {
-                const int n = tc.tn * BN + j;
-                const bool in = n < P.N;
-                sw_s[j] = in ? __ldg(P.sw + n) : 0.0f;
-                b_s[j] = (in && P.bias != nullptr) ? __uint_as_float((uint32_t)__ldg(P.bias + n) << 16) : 0.0f;
+#pragma unroll
+            for (int i = 0; i < SW_V4; ++i) {
+                const int n = tc.tn * BN + (i * 32 + lane) * 4;
+                p.sw[i] = n < P.N ? __ldg(reinterpret_cast<const float4*>(P.sw + n)) : make_float4(0, 0, 0, 0);
             }
+#pragma unroll
+            for (int i = 0; i < B_V8; ++i) {
+                const int v = i * 32 + lane;
+                const int n = tc.tn * BN + v * 8;
+                p.b[i] = (v < BN / 8 && n < P.N && P.bias != nullptr)
+                             ? __ldg(reinterpret_cast<const uint4*>(P.bias + n))
+                             : make_uint4(0, 0, 0, 0);
+            }
+            const int row = tc.tm * C::BM + (int)rank * C::ROWS + q * 32 + lane;
+            p.sa = row < args.M ? __ldg(args.sa + row) : 0.0f;
+        };
+        auto publish = [&](const Pre& p) {  // this warp's smem copy of sw / bias (fp32)
+#pragma unroll
+            for (int i = 0; i < SW_V4; ++i) *reinterpret_cast<float4*>(sw_s + (i * 32 + lane) * 4) = p.sw[i];
+#pragma unroll
+            for (int i = 0; i < B_V8; ++i) {
+                if (i * 32 + lane >= BN / 8) break;
+                const uint32_t w[4] = {p.b[i].x, p.b[i].y, p.b[i].z, p.b[i].w};
+                float* dst = b_s + (i * 32 + lane) * 8;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    dst[2 * k] = __uint_as_float(w[k] << 16);
+                    dst[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+                }
+            }
+        };
+
+        uint32_t acc = 0, acc_phase = 0;
+        uint32_t stores = 0;
+        Pre pre;
+        if (unit < args.num_tiles) fetch(unit, pre);
+        for (int t = unit; t < args.num_tiles; t += units) {
+            const TileCoord tc = tile_coord(args, t);
+            __syncwarp();  // every lane is done reading the previous tile's copy
+            publish(pre);
+            const float sa = pre.sa;
             __syncwarp();
+            if (t + units < args.num_tiles) fetch(t + units, pre);
             const int row0 = tc.tm * C::BM + (int)rank * C::ROWS + q * 32;  // first row of this warp's box
-            const int row = row0 + lane;
-            const float sa = row < args.M ? __ldg(args.sa + row) : 0.0f;
 
             // Every lane waits; the warp then agrees (and reconverges) before
             // the warp-collective TMEM loads.
@@ -272,11 +314,12 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
                 break;
             }
             tc_fence_after();
+            const int n_tile = args.prob[tc.g].N;
             const uint32_t t_addr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 const int n0 = tc.tn * BN + c * 32;
-                if (n0 >= P.N) break;  // warp-uniform
+                if (n0 >= n_tile) break;  // warp-uniform
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_addr + c * 32, r);
                 tmem_wait_ld();

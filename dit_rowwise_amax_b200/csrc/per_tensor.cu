@@ -14,12 +14,9 @@
 // are done. Chunks are claimed in queue order by running blocks, and amax
 // chunks never wait, so every wait is on work already held by a running
 // block: the launch cannot deadlock whatever the grid size.
-#include <cuda_bf16.h>
-#include <cuda_fp8.h>
+#include <algorithm>
 
-#include <vector>
-
-#include "fp8dit_internal.cuh"
+#include "fp8_codec.cuh"
 
 namespace fp8dit {
 namespace {
@@ -40,19 +37,6 @@ struct PerTensorArgs {
     DevErr err;
 };
 
-template <int FMT>
-struct Fmt;
-template <>
-struct Fmt<FP8DIT_E4M3FN> {
-    static constexpr float kMax = 448.0f;
-    static constexpr __nv_fp8_interpretation_t kInterp = __NV_E4M3;
-};
-template <>
-struct Fmt<FP8DIT_E5M2> {
-    static constexpr float kMax = 57344.0f;
-    static constexpr __nv_fp8_interpretation_t kInterp = __NV_E5M2;
-};
-
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -62,36 +46,11 @@ __device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t w, uint32_t acc) {
-    __nv_bfloat162 a, b;
-    uint32_t wm = w & 0x7fff7fffu;
-    *reinterpret_cast<uint32_t*>(&a) = acc;
-    *reinterpret_cast<uint32_t*>(&b) = wm;
-    a = __hmax2(a, b);
-    return *reinterpret_cast<uint32_t*>(&a);
-}
-
-template <int FMT>
-__device__ __forceinline__ uint32_t quant2(uint32_t w, float s) {
-    const float lo = __uint_as_float(w << 16);
-    const float hi = __uint_as_float(w & 0xffff0000u);
-    float2 qf = make_float2(__fdiv_rn(lo, s), __fdiv_rn(hi, s));
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(qf, __NV_SATFINITE, Fmt<FMT>::kInterp);
-}
-
-template <int FMT>
-__device__ __forceinline__ uint8_t quant1(uint16_t b, float s) {
-    const float f = __uint_as_float((uint32_t)b << 16);
-    return (uint8_t)(__nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f, s), 0.0f), __NV_SATFINITE,
-                                              Fmt<FMT>::kInterp) &
-                     0xffu);
-}
-
 template <int FMT>
 __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_constant__ PerTensorArgs a) {
     __shared__ unsigned long long s_item;
     __shared__ uint32_t s_red[kThreads / 32];
-    __shared__ float s_scale;
+    __shared__ float s_amax;
     __shared__ int s_ok;
     const unsigned long long total = (unsigned long long)a.stage_start[a.n + 1];
 
@@ -126,16 +85,12 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
             for (int i = 0; i < kVecPerThread; ++i) {
                 const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
                 if (vi < nvec) {
-                    const uint4 v = __ldg(src + vi);
-                    packed = absmax_bf16x2(v.x, packed);
-                    packed = absmax_bf16x2(v.y, packed);
-                    packed = absmax_bf16x2(v.z, packed);
-                    packed = absmax_bf16x2(v.w, packed);
+                    packed = absmax8(__ldg(src + vi), packed);
                 }
             }
             for (int64_t e = begin + nvec * 8 + threadIdx.x; e < end; e += kThreads)
-                packed = absmax_bf16x2((uint32_t)d.src[e], packed);
-            uint32_t m = max(packed & 0xffffu, packed >> 16);
+                packed = absmax2((uint32_t)d.src[e], packed);
+            uint32_t m = fold_halves(packed);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
@@ -165,33 +120,27 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
                         }
                     }
                 }
-                const uint32_t bits = ld_acquire_gpu(&a.amax_bits[t]);
-                const float amax = __uint_as_float(bits << 16);
-                const float s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, Fmt<FMT>::kMax);
-                s_scale = s;
+                const float amax = bf16_bits_to_float(ld_acquire_gpu(&a.amax_bits[t]));
+                s_amax = amax;
                 s_ok = ok;
-                if (ok && chunk == 0) *d.scale = s;
+                if (ok && chunk == 0) *d.scale = scale_ctx<FMT>(amax).s;
             }
             __syncthreads();
             if (s_ok) {
-                const float s = s_scale;
+                const ScaleCtx c = scale_ctx<FMT>(s_amax);
                 uint8_t* dst = d.dst + begin;
 #pragma unroll 4
                 for (int i = 0; i < kVecPerThread; ++i) {
                     const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
                     if (vi < nvec) {
-                        const uint4 v = __ldcs(src + vi);
-                        uint2 o;
-                        o.x = quant2<FMT>(v.x, s) | (quant2<FMT>(v.y, s) << 16);
-                        o.y = quant2<FMT>(v.z, s) | (quant2<FMT>(v.w, s) << 16);
-                        __stcs(reinterpret_cast<uint2*>(dst) + vi, o);
+                        __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT>(__ldcs(src + vi), c));
                     }
                 }
                 for (int64_t e = begin + nvec * 8 + threadIdx.x; e < end; e += kThreads)
-                    d.dst[e] = quant1<FMT>(d.src[e], s);
+                    d.dst[e] = quant1<FMT>(d.src[e], c);
             }
         }
-        __syncthreads();  // s_item / s_red / s_scale are rewritten next iteration
+        __syncthreads();  // s_item / s_red / s_amax are rewritten next iteration
     }
 }
 

@@ -3,134 +3,95 @@
 // Recipe ("ComfyUI自定义节点开发适配Stable Diffusion 3.5 FP8技术要点", section
 // "FP8：不只是精度减半", steps 1-3, read for FP8): amax = max |x| over the row,
 // S = amax / fmax (IEEE fp32 division; S = 1 for an all-zero row),
-// q = RNE-saturating FP8 of the IEEE fp32 quotient x / S. Applied per token
-// to activations ("从 BF16 到 FP8：HunyuanVideo1.5推理优化复盘", section 三.1)
-// and per output channel to weights (section 二).
+// q = RNE-saturating FP8 of the fp32 quotient x / S. Applied per token to
+// activations ("从 BF16 到 FP8：HunyuanVideo1.5推理优化复盘", section 三.1) and per
+// output channel to weights (section 二).
 //
 // Design: the op is HBM-bound (2 B read + 1 B written per element). A group
 // of TPR threads owns one row and holds it in registers (VPT 16-byte vectors
 // per thread, coalesced across the group), so each element is read from HBM
-// exactly once: load -> packed bf16 |max| -> shuffle / shared-memory max across
-// the group -> scale -> divide, convert two at a time with
-// cvt.rn.satfinite.{e4m3x2,e5m2x2}.f32 -> 8-byte stores. Rows longer than
+// once: load -> packed bf16 |max| -> shuffle / shared-memory max across the
+// group -> scale and reciprocal -> corrected-reciprocal quotient -> convert
+// two at a time -> 8-byte stores. Blocks are persistent (grid = resident
+// blocks) and load the next row group's vectors before quantising the
+// current one, so HBM reads overlap the arithmetic. Rows longer than
 // 256 threads x 4 vectors x 8 = 8192 elements take a two-pass kernel whose
 // second read of the row comes from L2.
-#include <cuda_bf16.h>
-#include <cuda_fp8.h>
+#include <algorithm>
 
-#include "fp8dit_internal.cuh"
+#include "fp8_codec.cuh"
 
 namespace fp8dit {
 namespace {
 
-template <int FMT>
-struct Fmt;
-template <>
-struct Fmt<FP8DIT_E4M3FN> {
-    static constexpr float kMax = 448.0f;
-    static constexpr __nv_fp8_interpretation_t kInterp = __NV_E4M3;
-};
-template <>
-struct Fmt<FP8DIT_E5M2> {
-    static constexpr float kMax = 57344.0f;
-    static constexpr __nv_fp8_interpretation_t kInterp = __NV_E5M2;
-};
-
-__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t u) {
-    __nv_bfloat162 r;
-    *reinterpret_cast<uint32_t*>(&r) = u;
-    return r;
-}
-__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
-
-// Running packed max of |bf16| over the 8 values of a 16-byte vector.
-__device__ __forceinline__ uint32_t absmax8(const uint4& v, uint32_t acc) {
-    __nv_bfloat162 m = as_bf162(acc);
-    m = __hmax2(m, as_bf162(v.x & 0x7fff7fffu));
-    m = __hmax2(m, as_bf162(v.y & 0x7fff7fffu));
-    m = __hmax2(m, as_bf162(v.z & 0x7fff7fffu));
-    m = __hmax2(m, as_bf162(v.w & 0x7fff7fffu));
-    return as_u32(m);
-}
-
-// Larger of the two non-negative bf16 halves, as its 16-bit pattern.
-__device__ __forceinline__ uint32_t fold_halves(uint32_t packed) {
-    return max(packed & 0xffffu, packed >> 16);
-}
-
-template <int FMT>
-__device__ __forceinline__ float scale_of(uint32_t amax_bits) {
-    const float amax = __uint_as_float(amax_bits << 16);
-    return amax == 0.0f ? 1.0f : __fdiv_rn(amax, Fmt<FMT>::kMax);
-}
-
-// Two bf16 (one 32-bit word) -> two FP8 codes (low byte = low element).
-template <int FMT>
-__device__ __forceinline__ uint32_t quant2(uint32_t w, float s) {
-    const float lo = __uint_as_float(w << 16);
-    const float hi = __uint_as_float(w & 0xffff0000u);
-    float2 qf = make_float2(__fdiv_rn(lo, s), __fdiv_rn(hi, s));
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(qf, __NV_SATFINITE, Fmt<FMT>::kInterp);
-}
-
-template <int FMT>
-__device__ __forceinline__ uint2 quant8(const uint4& v, float s) {
-    uint2 o;
-    o.x = quant2<FMT>(v.x, s) | (quant2<FMT>(v.y, s) << 16);
-    o.y = quant2<FMT>(v.z, s) | (quant2<FMT>(v.w, s) << 16);
-    return o;
-}
-
 constexpr int kThreads = 256;
 
-// TPR threads per row (power of two, 8..256), VPT 16-byte vectors per thread.
-template <int TPR, int VPT, int FMT>
-__global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* __restrict__ x, int64_t M,
-                                                                 int32_t K, int64_t ldx, uint8_t* __restrict__ q,
-                                                                 int64_t ldq, float* __restrict__ scale) {
+template <int TPR, int VPT>
+__device__ __forceinline__ void load_group(const uint16_t* __restrict__ x, int64_t M, int nvec, int64_t ldx,
+                                           int64_t g, uint4 (&v)[VPT]) {
     constexpr int RPB = kThreads / TPR;
     const int t = threadIdx.x % TPR;
-    const int r = threadIdx.x / TPR;
-    const int64_t row = (int64_t)blockIdx.x * RPB + r;
+    const int64_t row = g * RPB + threadIdx.x / TPR;
     const bool active = row < M;
-    const int nvec = K >> 3;
     const uint4* xr = reinterpret_cast<const uint4*>(x + (active ? row : 0) * ldx);
-
-    uint4 v[VPT];
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
         const int vi = i * TPR + t;
         v[i] = (active && vi < nvec) ? __ldcs(xr + vi) : make_uint4(0, 0, 0, 0);
     }
-    uint32_t packed = 0;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) packed = absmax8(v[i], packed);
-    uint32_t m = fold_halves(packed);
+}
 
-    if constexpr (TPR <= 32) {
-#pragma unroll
-        for (int off = TPR / 2; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-    } else {
-        constexpr int WPR = TPR / 32;  // warps per row
-        __shared__ uint32_t red[kThreads / 32];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-        __syncthreads();
-        m = red[r * WPR];
-#pragma unroll
-        for (int w = 1; w < WPR; ++w) m = max(m, red[r * WPR + w]);
-    }
-    const float s = scale_of<FMT>(m);
-    if (!active) return;
+// TPR threads per row (power of two, 8..256), VPT 16-byte vectors per thread.
+template <int TPR, int VPT, int FMT>
+__global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* __restrict__ x, int64_t M,
+                                                                 int32_t K, int64_t ldx, uint8_t* __restrict__ q,
+                                                                 int64_t ldq, float* __restrict__ scale,
+                                                                 int64_t groups) {
+    constexpr int RPB = kThreads / TPR;
+    constexpr int WPR = TPR / 32;  // warps per row (when TPR >= 32)
+    __shared__ uint32_t red[2][kThreads / 32];
+    const int t = threadIdx.x % TPR;
+    const int r = threadIdx.x / TPR;
+    const int nvec = K >> 3;
 
-    uint8_t* qr = q + row * ldq;
+    uint4 cur[VPT], nxt[VPT];
+    int64_t g = blockIdx.x;
+    load_group<TPR, VPT>(x, M, nvec, ldx, g, cur);
+    for (int it = 0; g < groups; g += gridDim.x, ++it) {
+        const int64_t gn = g + gridDim.x;
+        if (gn < groups) load_group<TPR, VPT>(x, M, nvec, ldx, gn, nxt);
+
+        uint32_t packed = 0;
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-        const int vi = i * TPR + t;
-        if (vi < nvec) *reinterpret_cast<uint2*>(qr + (int64_t)vi * 8) = quant8<FMT>(v[i], s);
+        for (int i = 0; i < VPT; ++i) packed = absmax8(cur[i], packed);
+        uint32_t m = fold_halves(packed);
+        if constexpr (TPR <= 32) {
+#pragma unroll
+            for (int off = TPR / 2; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        } else {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+            uint32_t* rb = red[it & 1];  // alternate buffers: no second barrier per group
+            if ((threadIdx.x & 31) == 0) rb[threadIdx.x >> 5] = m;
+            __syncthreads();
+            m = rb[r * WPR];
+#pragma unroll
+            for (int w = 1; w < WPR; ++w) m = max(m, rb[r * WPR + w]);
+        }
+        const ScaleCtx c = scale_ctx<FMT>(bf16_bits_to_float(m));
+        const int64_t row = g * RPB + r;
+        if (row < M) {
+            uint8_t* qr = q + row * ldq;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int vi = i * TPR + t;
+                if (vi < nvec) *reinterpret_cast<uint2*>(qr + (int64_t)vi * 8) = quant8<FMT>(cur[i], c);
+            }
+            if (t == 0) scale[row] = c.s;
+        }
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) cur[i] = nxt[i];
     }
-    if (t == 0) scale[row] = s;
 }
 
 // One block per row (grid-strided): amax pass, then a quantise pass that
@@ -155,22 +116,29 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_
 #pragma unroll
         for (int w = 1; w < kThreads / 32; ++w) m = max(m, red[w]);
         __syncthreads();  // red is reused by the next row
-        const float s = scale_of<FMT>(m);
+        const ScaleCtx c = scale_ctx<FMT>(bf16_bits_to_float(m));
         uint8_t* qr = q + row * ldq;
         for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads)
-            *reinterpret_cast<uint2*>(qr + vi * 8) = quant8<FMT>(__ldcs(xr + vi), s);
-        if (threadIdx.x == 0) scale[row] = s;
+            *reinterpret_cast<uint2*>(qr + vi * 8) = quant8<FMT>(__ldcs(xr + vi), c);
+        if (threadIdx.x == 0) scale[row] = c.s;
     }
 }
 
 template <int TPR, int VPT, int FMT>
 cudaError_t launch_regs(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
-                        float* scale, cudaStream_t stream) {
+                        float* scale, cudaStream_t stream, const DeviceInfo* dev) {
     constexpr int RPB = kThreads / TPR;
-    const int64_t blocks = (M + RPB - 1) / RPB;
-    if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    quantize_rows_regs<TPR, VPT, FMT><<<(unsigned)blocks, kThreads, 0, stream>>>(x, M, (int32_t)K, ldx, q, ldq,
-                                                                                  scale);
+    static int per_sm = 0;  // resident blocks per SM (same on every sm_100a device)
+    if (per_sm == 0) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_rows_regs<TPR, VPT, FMT>,
+                                                                       kThreads, 0);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+    }
+    const int64_t groups = (M + RPB - 1) / RPB;
+    const int64_t grid = std::min<int64_t>(groups, (int64_t)dev->num_sms * per_sm);
+    quantize_rows_regs<TPR, VPT, FMT><<<(unsigned)grid, kThreads, 0, stream>>>(x, M, (int32_t)K, ldx, q, ldq,
+                                                                                scale, groups);
     return cudaGetLastError();
 }
 
@@ -189,8 +157,8 @@ cudaError_t launch_fmt(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uin
     const bool two = nvec <= tpr * 2;
 #define FP8DIT_Q_CASE(T)                                                                        \
     case T:                                                                                     \
-        return two ? launch_regs<T, 2, FMT>(x, M, K, ldx, q, ldq, scale, stream)                \
-                   : launch_regs<T, 4, FMT>(x, M, K, ldx, q, ldq, scale, stream);
+        return two ? launch_regs<T, 2, FMT>(x, M, K, ldx, q, ldq, scale, stream, dev)           \
+                   : launch_regs<T, 4, FMT>(x, M, K, ldx, q, ldq, scale, stream, dev);
     switch (tpr) {
         FP8DIT_Q_CASE(8)
         FP8DIT_Q_CASE(16)
@@ -204,6 +172,31 @@ cudaError_t launch_fmt(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uin
 #undef FP8DIT_Q_CASE
 }
 
+// Exhaustive comparison of the quantiser's quotient path with IEEE division:
+// thread i takes amax = bf16 pattern (i + 1) and walks every bf16 x with
+// |x| <= amax (both signs), counting FP8 code mismatches per format.
+__global__ void selftest_quotient_kernel(unsigned long long* mismatch) {
+    const uint32_t amax_bits = blockIdx.x * blockDim.x + threadIdx.x + 1;
+    if (amax_bits > 0x7F7Fu) return;
+    const float amax = bf16_bits_to_float(amax_bits);
+    const ScaleCtx c4 = scale_ctx<FP8DIT_E4M3FN>(amax);
+    const ScaleCtx c5 = scale_ctx<FP8DIT_E5M2>(amax);
+    unsigned long long bad4 = 0, bad5 = 0;
+    for (uint32_t mag = 0; mag <= amax_bits; ++mag) {
+        for (uint32_t sign = 0; sign < 2; ++sign) {
+            const float xv = bf16_bits_to_float(mag | (sign << 15));
+            const float f4 = quotient(xv, c4), r4 = __fdiv_rn(xv, c4.s);
+            const float f5 = quotient(xv, c5), r5 = __fdiv_rn(xv, c5.s);
+            const uint32_t a4 = __nv_cvt_float2_to_fp8x2(make_float2(f4, r4), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t a5 = __nv_cvt_float2_to_fp8x2(make_float2(f5, r5), __NV_SATFINITE, __NV_E5M2);
+            bad4 += (a4 & 0xffu) != (a4 >> 8);
+            bad5 += (a5 & 0xffu) != (a5 >> 8);
+        }
+    }
+    if (bad4) atomicAdd(&mismatch[0], bad4);
+    if (bad5) atomicAdd(&mismatch[1], bad5);
+}
+
 }  // namespace
 
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int fmt, uint8_t* q,
@@ -211,6 +204,13 @@ cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_
     if (M == 0) return cudaSuccess;
     return fmt == FP8DIT_E4M3FN ? launch_fmt<FP8DIT_E4M3FN>(x, M, K, ldx, q, ldq, scale, stream, dev)
                                 : launch_fmt<FP8DIT_E5M2>(x, M, K, ldx, q, ldq, scale, stream, dev);
+}
+
+cudaError_t launch_selftest_quotient(unsigned long long* mismatch, cudaStream_t stream) {
+    const int threads = 128;
+    const int blocks = (0x7F7F + threads - 1) / threads;
+    selftest_quotient_kernel<<<blocks, threads, 0, stream>>>(mismatch);
+    return cudaGetLastError();
 }
 
 }  // namespace fp8dit

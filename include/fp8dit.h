@@ -97,7 +97,7 @@ fp8dit_status fp8_quantize_weight_per_channel(const uint16_t* w, int64_t N, int6
 /* One tensor of a per-tensor conversion. Pointers are device pointers. */
 typedef struct {
     const uint16_t* src; /* numel bf16 values, contiguous, 16-byte aligned */
-    int64_t numel;       /* >= 0; numel % 8 == 0 */
+    int64_t numel;       /* >= 0, any size */
     uint8_t* dst;        /* numel FP8 codes, 16-byte aligned */
     float* scale;        /* one fp32: S of the tensor (left untouched when numel == 0) */
 } fp8dit_tensor_desc;
@@ -132,7 +132,7 @@ fp8dit_status fp8_quantize_weight_per_tensor(const fp8dit_tensor_desc* tensors, 
  *   bias [N] bf16, or NULL for no bias.
  * The handle BORROWS qw, sw and bias: they must stay valid and unchanged
  * until fp8_linear_destroy. device is the CUDA device that holds them.
- * Requires N % 8 == 0, K % 16 == 0, qw 16-byte aligned.
+ * Requires N % 8 == 0, K % 16 == 0; qw, sw and bias 16-byte aligned.
  */
 fp8dit_status fp8_linear_create(int64_t N, int64_t K, const uint8_t* qw, const float* sw,
                                 const uint16_t* bias, int device, fp8dit_linear* out);
@@ -192,6 +192,16 @@ fp8dit_status fp8dit_device_error(fp8dit_stream_t stream);
  * failure path without faulting the GPU.
  */
 fp8dit_status fp8dit_selftest_expired_wait(int64_t limit_ns, fp8dit_stream_t stream);
+
+/*
+ * Exhaustive check of the quantisers' quotient arithmetic: for every finite
+ * positive bf16 amax and every bf16 x with |x| <= amax, the FP8 code the
+ * quantisers produce for x / S (S = amax / fmax) is compared with the code of
+ * the IEEE fp32 division x / S, for E4M3FN and E5M2. Adds the number of
+ * differing codes to mismatch[0] (E4M3FN) and mismatch[1] (E5M2), a DEVICE
+ * array of two uint64 the caller zeroes. Asynchronous on `stream`.
+ */
+fp8dit_status fp8dit_selftest_quotient(unsigned long long* mismatch, fp8dit_stream_t stream);
 
 /* Description of the last failure on this thread ("" if none). */
 const char* fp8dit_last_error_string(void);

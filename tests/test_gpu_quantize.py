@@ -123,3 +123,9 @@ def test_zero_rows_is_noop():
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     q, s = fp8.quantize_rowwise(x)
     assert q.shape == (0, 64) and s.shape == (0,)
+
+
+def test_quotient_selftest_exhaustive():
+    """Every (bf16 x, bf16 amax) pair, both formats: the quantisers' quotient
+    path gives the same FP8 code as IEEE fp32 division (hardware cvt)."""
+    assert fp8.selftest_quotient() == (0, 0)
