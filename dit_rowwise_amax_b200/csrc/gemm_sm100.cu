@@ -14,11 +14,12 @@
 //   warp 1      allocates TMEM; one thread of the pair's leader CTA issues
 //               tcgen05.mma (K = 32 per instruction) into a TMEM accumulator
 //               and commits each ring slot back to the producers;
-//   warps 2..5  epilogue: fetch the next tile's sw / bias / sa while this
-//               tile is processed, tcgen05.ld 32 accumulator columns at a
-//               time, scale, bias,
-//               bf16, write a 32 x 32 box into a 64-byte-swizzled staging
-//               buffer and TMA-store it (double-buffered per warp).
+//   warps 2..9  epilogue, two warps per TMEM lane quarter, each taking half
+//               of the tile's columns: fetch the next tile's sw / bias / sa
+//               while this tile is processed, tcgen05.ld 32 accumulator
+//               columns at a time, scale, bias, bf16, write a 32 x 32 box
+//               into the warp's 64-byte-swizzled staging buffer and
+//               TMA-store it.
 // Two TMEM accumulators let the epilogue of tile i overlap the mainloop of
 // tile i+1.
 //
@@ -51,15 +52,16 @@ struct Cfg {
     static constexpr int STAGES = (CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6);
     static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
-    static constexpr int EPI_WARPS = 4;
+    static constexpr int EPI_WARPS = 8;              // two per TMEM lane quarter, each half the columns
+    static constexpr int EPI_COLS = BN / 2;          // columns per epilogue warp
     static constexpr int BOX = 32;                   // epilogue store box: 32 rows x 32 columns
-    static constexpr int STG_BYTES = BOX * BOX * 2;  // 2 KB, 64-byte rows
-    static constexpr int STAGING_BYTES = EPI_WARPS * 2 * STG_BYTES;
-    static constexpr int SWB_FLOATS = 2 * BN;        // sw then bias as fp32, one copy per epilogue warp
+    static constexpr int STG_BYTES = BOX * BOX * 2;  // 2 KB, 64-byte rows, one per epilogue warp
+    static constexpr int STAGING_BYTES = EPI_WARPS * STG_BYTES;
+    static constexpr int SWB_FLOATS = 2 * EPI_COLS;  // sw then bias as fp32, one copy per epilogue warp
     static constexpr int SWB_BYTES = EPI_WARPS * SWB_FLOATS * 4;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
     static_assert((2 * STAGES + 2 * ACC + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -241,16 +243,17 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps
-        const int q = warp & 3;     // TMEM lane quarter this warp may access
-        const int ew = warp - 2;    // this warp's staging buffers and scale copy
-        uint8_t* stg = staging + ew * 2 * C::STG_BYTES;
+        const int q = warp & 3;          // TMEM lane quarter this warp may access
+        const int ew = warp - 2;         // 0..7
+        const int col0 = (ew >> 2) * C::EPI_COLS;  // this warp's half of the tile's columns
+        uint8_t* stg = staging + ew * C::STG_BYTES;
         float* sw_s = swb + ew * C::SWB_FLOATS;
-        float* b_s = sw_s + BN;
-        constexpr int SW_V4 = BN / 4 / 32;  // float4 of sw per lane
-        constexpr int B_V8 = (BN / 8 + 31) / 32;  // 8-wide bf16 bias vectors per lane (lanes >= BN/8 idle)
+        float* b_s = sw_s + C::EPI_COLS;
+        constexpr int SW_V4 = (C::EPI_COLS / 4 + 31) / 32;  // float4 of sw per lane
+        constexpr int B_V8 = (C::EPI_COLS / 8 + 31) / 32;   // 8-wide bf16 bias vectors per lane
 
         // Per-tile epilogue operands, fetched one tile ahead: the scales and
-        // bias of the tile's columns, and sa of this lane's row. All loads of
+        // bias of this warp's columns, and sa of this lane's row. All loads of
         // a tile are independent, so one memory round trip covers them, and
         // it overlaps the previous tile's processing.
         struct Pre {
@@ -263,14 +266,16 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
             const GemmProblem& P = args.prob[tc.g];
 #pragma unroll
             for (int i = 0; i < SW_V4; ++i) {
-                const int n = tc.tn * BN + (i * 32 + lane) * 4;
-                p.sw[i] = n < P.N ? __ldg(reinterpret_cast<const float4*>(P.sw + n)) : make_float4(0, 0, 0, 0);
+                const int v = i * 32 + lane;
+                const int n = tc.tn * BN + col0 + v * 4;
+                p.sw[i] = (v < C::EPI_COLS / 4 && n < P.N) ? __ldg(reinterpret_cast<const float4*>(P.sw + n))
+                                                            : make_float4(0, 0, 0, 0);
             }
 #pragma unroll
             for (int i = 0; i < B_V8; ++i) {
                 const int v = i * 32 + lane;
-                const int n = tc.tn * BN + v * 8;
-                p.b[i] = (v < BN / 8 && n < P.N && P.bias != nullptr)
+                const int n = tc.tn * BN + col0 + v * 8;
+                p.b[i] = (v < C::EPI_COLS / 8 && n < P.N && P.bias != nullptr)
                              ? __ldg(reinterpret_cast<const uint4*>(P.bias + n))
                              : make_uint4(0, 0, 0, 0);
             }
@@ -279,10 +284,13 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
         };
         auto publish = [&](const Pre& p) {  // this warp's smem copy of sw / bias (fp32)
 #pragma unroll
-            for (int i = 0; i < SW_V4; ++i) *reinterpret_cast<float4*>(sw_s + (i * 32 + lane) * 4) = p.sw[i];
+            for (int i = 0; i < SW_V4; ++i) {
+                if (i * 32 + lane >= C::EPI_COLS / 4) break;
+                *reinterpret_cast<float4*>(sw_s + (i * 32 + lane) * 4) = p.sw[i];
+            }
 #pragma unroll
             for (int i = 0; i < B_V8; ++i) {
-                if (i * 32 + lane >= BN / 8) break;
+                if (i * 32 + lane >= C::EPI_COLS / 8) break;
                 const uint32_t w[4] = {p.b[i].x, p.b[i].y, p.b[i].z, p.b[i].w};
                 float* dst = b_s + (i * 32 + lane) * 8;
 #pragma unroll
@@ -315,10 +323,10 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
             }
             tc_fence_after();
             const int n_tile = args.prob[tc.g].N;
-            const uint32_t t_addr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+            const uint32_t t_addr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + col0;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                const int n0 = tc.tn * BN + c * 32;
+            for (int c = 0; c < C::EPI_COLS / 32; ++c) {
+                const int n0 = tc.tn * BN + col0 + c * 32;
                 if (n0 >= n_tile) break;  // warp-uniform
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_addr + c * 32, r);
@@ -335,22 +343,22 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
                     packed[j / 2] = pack_bf16x2(o0, o1);
                     packed[j / 2 + 1] = pack_bf16x2(o2, o3);
                 }
-                uint8_t* buf = stg + (stores & 1u) * C::STG_BYTES;
-                if (stores >= 2) {
-                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last used `buf` has read it
+                // The single staging buffer is free once the previous store has read it.
+                if (stores >= 1) {
+                    if (lane == 0) bulk_wait_group_read<0>();
                     __syncwarp();
                 }
                 // Row `lane` of a 32 x 32 bf16 box, 64-byte rows, 64-byte swizzle.
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
                     const int phys = k4 ^ ((lane >> 1) & 3);
-                    *reinterpret_cast<uint4*>(buf + lane * 64 + phys * 16) =
+                    *reinterpret_cast<uint4*>(stg + lane * 64 + phys * 16) =
                         make_uint4(packed[4 * k4], packed[4 * k4 + 1], packed[4 * k4 + 2], packed[4 * k4 + 3]);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && row0 < args.M) {
-                    tma_store_2d(&args.tmY[tc.g], buf, n0, row0);
+                    tma_store_2d(&args.tmY[tc.g], stg, n0, row0);
                     bulk_commit_group();
                 }
                 ++stores;
