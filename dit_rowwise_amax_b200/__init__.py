@@ -73,6 +73,7 @@ def load_library():
     L.fp8_linear_destroy.argtypes = [p]
     L.fp8_scaled_linear.argtypes = [p, i64, p, p, p, p, p, p, p]
     L.fp8_scaled_linear_multi.argtypes = [ctypes.POINTER(p), i32, i64, p, p, p, ctypes.POINTER(p), p]
+    L.fp8_scaled_linear_noalloc.argtypes = [p, i64, p, p, p]
     L.fp8_linear_plan.argtypes = [p, i64, i32, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.fp8dit_device_error.argtypes = [p]
     L.fp8dit_selftest_expired_wait.argtypes = [i64, p]
@@ -80,6 +81,7 @@ def load_library():
     L.fp8dit_last_error_string.restype = ctypes.c_char_p
     for name in ("fp8_quantize_rowwise", "fp8_quantize_weight_per_channel", "fp8_quantize_weight_per_tensor",
                  "fp8_linear_create", "fp8_linear_destroy", "fp8_scaled_linear", "fp8_scaled_linear_multi",
+                 "fp8_scaled_linear_noalloc",
                  "fp8_linear_plan", "fp8dit_device_error", "fp8dit_selftest_expired_wait",
                  "fp8dit_selftest_quotient"):
         getattr(L, name).restype = st

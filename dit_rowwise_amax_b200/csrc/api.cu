@@ -162,6 +162,8 @@ struct fp8dit_linear_s {
     CUtensorMap tmB[kNumCfgs];  // weight descriptors, one per tile configuration
 };
 
+int64_t fp8dit::linear_k(const fp8dit_linear_s* h) { return h->K; }
+
 static int64_t tiles_for(const fp8dit_linear_s* h, int64_t M, int n_problems, int cfg) {
     const int64_t bm = gemm_block_m(cfg), bn = gemm_block_n(cfg);
     return ((M + bm - 1) / bm) * ((h->N + bn - 1) / bn) * n_problems;

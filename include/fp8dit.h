@@ -156,6 +156,30 @@ fp8dit_status fp8_scaled_linear(fp8dit_linear h, int64_t M, const uint16_t* a_bf
                                 float* sa_scratch, uint16_t* y, fp8dit_stream_t stream);
 
 /*
+ * fp8_scaled_linear from a bf16 activation, for callers that cannot allocate
+ * device memory. The pages have no counterpart: this entry exists for code
+ * that has no way to hand the library qa / sa scratch, such as a plugin whose
+ * host framework owns the device allocator, or code that must not call
+ * cudaMalloc / cudaFree because they can synchronise the device and can fail
+ * for lack of memory mid-step. The quantised activation is kept in a fixed
+ * array that is part of the library's device image instead, so this call
+ * allocates nothing.
+ *   a_bf16 [M, K] bf16 contiguous, y [M, N] bf16 contiguous, both 16-byte
+ *   aligned; results equal fp8_scaled_linear(h, M, a_bf16, NULL, NULL, ...).
+ * Limits: M <= FP8DIT_NOALLOC_MAX_ROWS and M * K <= FP8DIT_NOALLOC_MAX_ACT_BYTES;
+ * larger calls return FP8DIT_ERR_UNSUPPORTED_SHAPE and enqueue nothing.
+ * Every GPU that loads the library holds the array (about 8.25 MiB) until the
+ * process exits. All calls on a device share it and leave their data in it;
+ * each call rewrites everything it reads, but calls whose work overlaps on the
+ * GPU (e.g. on two streams) race. The first call on a device looks up the
+ * array's device address; make that call before any stream capture.
+ */
+#define FP8DIT_NOALLOC_MAX_ACT_BYTES (8u << 20)
+#define FP8DIT_NOALLOC_MAX_ROWS 65536
+fp8dit_status fp8_scaled_linear_noalloc(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, uint16_t* y,
+                                        fp8dit_stream_t stream);
+
+/*
  * n linear layers that read the same activation ("从 BF16 到 FP8", section
  * 三.4: quantise hidden_states once and feed the separate Q, K and V
  * projections). A [M, K] bf16 is quantised once into qa_scratch / sa_scratch,
