@@ -16,7 +16,8 @@
 // quotient (P. Markstein, "Computation of elementary functions on the IBM
 // RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990):
 //     q0 = RN(x R);   e = x - q0 S  (one FMA, exact);   q = RN(q0 + e R)
-// and the sign of x is restored for quotients that round to zero. This path
+// with the pair arithmetic done two lanes at a time (f32x2); each code takes
+// its sign bit from x, which also fixes the sign of zero quotients. This path
 // is taken only when amax >= 2^-64, so every x whose quotient can reach a
 // nonzero FP8 code is a normal fp32 number; smaller amax takes the IEEE
 // division. fp8dit_selftest_quotient() compares the resulting FP8 codes with
@@ -62,39 +63,85 @@ __device__ __forceinline__ ScaleCtx scale_ctx(float amax) {
     return c;
 }
 
-// RN_fp32(x / S).
-__device__ __forceinline__ float quotient(float x, const ScaleCtx& c) {
-    if (c.fast) {
-        const float q0 = __fmul_rn(x, c.r);
-        const float e = __fmaf_rn(-q0, c.s, x);
-        return copysignf(__fmaf_rn(e, c.r, q0), x);
-    }
-    return __fdiv_rn(x, c.s);
+// ---- packed fp32 pairs (sm_100a f32x2 arithmetic; each lane is an IEEE
+// round-to-nearest multiply or fused multiply-add).
+typedef unsigned long long f32x2_t;
+__device__ __forceinline__ f32x2_t f2_pack(float lo, float hi) {
+    f32x2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(f32x2_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return make_float2(lo, hi);
+}
+__device__ __forceinline__ f32x2_t f2_mul(f32x2_t a, f32x2_t b) {
+    f32x2_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2_t f2_fma(f32x2_t a, f32x2_t b, f32x2_t c) {
+    f32x2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// The per-scale operands of the packed quotient: {R, R} and {-S, -S}.
+struct Quot2 {
+    f32x2_t r2, ns2;
+    float s;
+};
+__device__ __forceinline__ Quot2 quot2_of(const ScaleCtx& c) {
+    return Quot2{f2_pack(c.r, c.r), f2_pack(-c.s, -c.s), c.s};
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Two bf16 (one 32-bit word) -> two FP8 codes, low byte = low element.
-template <int FMT>
-__device__ __forceinline__ uint32_t quant2(uint32_t w, const ScaleCtx& c) {
-    const float2 qf = make_float2(quotient(bf16_lo(w), c), quotient(bf16_hi(w), c));
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(qf, __NV_SATFINITE, Fp8Fmt<FMT>::kInterp);
+// RN_fp32(x / S) for the two bf16 of w (low element first). FAST selects the
+// corrected-reciprocal quotient; the IEEE division otherwise. The sign of a
+// zero quotient may differ from x's; callers take the code's sign bit from x.
+template <bool FAST>
+__device__ __forceinline__ float2 quotient2(uint32_t w, const Quot2& q) {
+    if (FAST) {
+        const f32x2_t x2 = f2_pack(bf16_lo(w), bf16_hi(w));
+        const f32x2_t q0 = f2_mul(x2, q.r2);
+        const f32x2_t e = f2_fma(q0, q.ns2, x2);  // x - q0 S, exact
+        return f2_unpack(f2_fma(e, q.r2, q0));
+    }
+    return make_float2(__fdiv_rn(bf16_lo(w), q.s), __fdiv_rn(bf16_hi(w), q.s));
 }
 
-// Eight bf16 (16 bytes) -> eight FP8 codes (8 bytes).
-template <int FMT>
-__device__ __forceinline__ uint2 quant8(const uint4& v, const ScaleCtx& c) {
+// Two bf16 (one 32-bit word) -> two FP8 codes in the low 16 bits (low element first), sign bits not yet applied.
+template <int FMT, bool FAST>
+__device__ __forceinline__ uint32_t codes2(uint32_t w, const Quot2& q) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(quotient2<FAST>(w, q), __NV_SATFINITE, Fp8Fmt<FMT>::kInterp);
+}
+
+// Sign bits of the four bf16 in (w0, w1), placed in the sign bit of each code byte.
+__device__ __forceinline__ uint32_t signs4(uint32_t w0, uint32_t w1) {
+    return __byte_perm(w0, w1, 0x7531) & 0x80808080u;
+}
+
+// Eight bf16 (16 bytes) -> eight FP8 codes (8 bytes). Every code carries the
+// sign of its input (x / S has x's sign, and zero quotients encode as a zero
+// of that sign).
+template <int FMT, bool FAST>
+__device__ __forceinline__ uint2 quant8(const uint4& v, const Quot2& q) {
     uint2 o;
-    o.x = quant2<FMT>(v.x, c) | (quant2<FMT>(v.y, c) << 16);
-    o.y = quant2<FMT>(v.z, c) | (quant2<FMT>(v.w, c) << 16);
+    o.x = (codes2<FMT, FAST>(v.x, q) | (codes2<FMT, FAST>(v.y, q) << 16)) | signs4(v.x, v.y);
+    o.y = (codes2<FMT, FAST>(v.z, q) | (codes2<FMT, FAST>(v.w, q) << 16)) | signs4(v.z, v.w);
     return o;
 }
 
+// One bf16 -> one FP8 code (tails).
 template <int FMT>
 __device__ __forceinline__ uint8_t quant1(uint16_t b, const ScaleCtx& c) {
-    const float q = quotient(__uint_as_float((uint32_t)b << 16), c);
-    return (uint8_t)(__nv_cvt_float2_to_fp8x2(make_float2(q, 0.0f), __NV_SATFINITE, Fp8Fmt<FMT>::kInterp) & 0xffu);
+    const Quot2 q = quot2_of(c);
+    const uint32_t w = (uint32_t)b;
+    const uint32_t code = c.fast ? codes2<FMT, true>(w, q) : codes2<FMT, false>(w, q);
+    return (uint8_t)((code & 0xffu) | ((b >> 8) & 0x80u));
 }
 
 // Running packed max of |bf16| over 2 / 8 values (sign bits cleared, then a

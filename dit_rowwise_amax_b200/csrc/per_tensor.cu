@@ -128,12 +128,19 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
             __syncthreads();
             if (s_ok) {
                 const ScaleCtx c = scale_ctx<FMT>(s_amax);
+                const Quot2 q2 = quot2_of(c);
                 uint8_t* dst = d.dst + begin;
+                if (c.fast) {
 #pragma unroll 4
-                for (int i = 0; i < kVecPerThread; ++i) {
-                    const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
-                    if (vi < nvec) {
-                        __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT>(__ldcs(src + vi), c));
+                    for (int i = 0; i < kVecPerThread; ++i) {
+                        const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+                        if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT, true>(__ldcs(src + vi), q2));
+                    }
+                } else {
+#pragma unroll 4
+                    for (int i = 0; i < kVecPerThread; ++i) {
+                        const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+                        if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT, false>(__ldcs(src + vi), q2));
                     }
                 }
                 for (int64_t e = begin + nvec * 8 + threadIdx.x; e < end; e += kThreads)

@@ -81,11 +81,20 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* _
         const ScaleCtx c = scale_ctx<FMT>(bf16_bits_to_float(m));
         const int64_t row = g * RPB + r;
         if (row < M) {
+            const Quot2 q2 = quot2_of(c);
             uint8_t* qr = q + row * ldq;
+            if (c.fast) {
 #pragma unroll
-            for (int i = 0; i < VPT; ++i) {
-                const int vi = i * TPR + t;
-                if (vi < nvec) *reinterpret_cast<uint2*>(qr + (int64_t)vi * 8) = quant8<FMT>(cur[i], c);
+                for (int i = 0; i < VPT; ++i) {
+                    const int vi = i * TPR + t;
+                    if (vi < nvec) *reinterpret_cast<uint2*>(qr + (int64_t)vi * 8) = quant8<FMT, true>(cur[i], q2);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < VPT; ++i) {
+                    const int vi = i * TPR + t;
+                    if (vi < nvec) *reinterpret_cast<uint2*>(qr + (int64_t)vi * 8) = quant8<FMT, false>(cur[i], q2);
+                }
             }
             if (t == 0) scale[row] = c.s;
         }
@@ -117,9 +126,15 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_
         for (int w = 1; w < kThreads / 32; ++w) m = max(m, red[w]);
         __syncthreads();  // red is reused by the next row
         const ScaleCtx c = scale_ctx<FMT>(bf16_bits_to_float(m));
+        const Quot2 q2 = quot2_of(c);
         uint8_t* qr = q + row * ldq;
-        for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads)
-            *reinterpret_cast<uint2*>(qr + vi * 8) = quant8<FMT>(__ldcs(xr + vi), c);
+        if (c.fast) {
+            for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads)
+                *reinterpret_cast<uint2*>(qr + vi * 8) = quant8<FMT, true>(__ldcs(xr + vi), q2);
+        } else {
+            for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads)
+                *reinterpret_cast<uint2*>(qr + vi * 8) = quant8<FMT, false>(__ldcs(xr + vi), q2);
+        }
         if (threadIdx.x == 0) scale[row] = c.s;
     }
 }
@@ -172,27 +187,32 @@ cudaError_t launch_fmt(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uin
 #undef FP8DIT_Q_CASE
 }
 
-// Exhaustive comparison of the quantiser's quotient path with IEEE division:
-// thread i takes amax = bf16 pattern (i + 1) and walks every bf16 x with
-// |x| <= amax (both signs), counting FP8 code mismatches per format.
+// Exhaustive comparison of the quantisers' code path with IEEE division:
+// thread i takes amax = bf16 pattern (i + 1) and, for every bf16 magnitude
+// m <= amax, encodes the pair (+m, -m) exactly as the kernels do
+// (codes2 + signs4) and as cvt(x / S) with the IEEE division, counting
+// differing codes.
+template <int FMT>
+__device__ unsigned long long selftest_amax(uint32_t amax_bits) {
+    const ScaleCtx c = scale_ctx<FMT>(bf16_bits_to_float(amax_bits));
+    const Quot2 q = quot2_of(c);
+    unsigned long long bad = 0;
+    for (uint32_t mag = 0; mag <= amax_bits; ++mag) {
+        const uint32_t w = mag | ((mag | 0x8000u) << 16);
+        const uint32_t got = ((c.fast ? codes2<FMT, true>(w, q) : codes2<FMT, false>(w, q)) | signs4(w, 0u)) & 0xffffu;
+        const float2 ref = make_float2(__fdiv_rn(bf16_lo(w), c.s), __fdiv_rn(bf16_hi(w), c.s));
+        const uint32_t want = (uint32_t)__nv_cvt_float2_to_fp8x2(ref, __NV_SATFINITE, Fp8Fmt<FMT>::kInterp) & 0xffffu;
+        const uint32_t diff = got ^ want;
+        bad += ((diff & 0xffu) != 0) + ((diff >> 8) != 0);
+    }
+    return bad;
+}
+
 __global__ void selftest_quotient_kernel(unsigned long long* mismatch) {
     const uint32_t amax_bits = blockIdx.x * blockDim.x + threadIdx.x + 1;
     if (amax_bits > 0x7F7Fu) return;
-    const float amax = bf16_bits_to_float(amax_bits);
-    const ScaleCtx c4 = scale_ctx<FP8DIT_E4M3FN>(amax);
-    const ScaleCtx c5 = scale_ctx<FP8DIT_E5M2>(amax);
-    unsigned long long bad4 = 0, bad5 = 0;
-    for (uint32_t mag = 0; mag <= amax_bits; ++mag) {
-        for (uint32_t sign = 0; sign < 2; ++sign) {
-            const float xv = bf16_bits_to_float(mag | (sign << 15));
-            const float f4 = quotient(xv, c4), r4 = __fdiv_rn(xv, c4.s);
-            const float f5 = quotient(xv, c5), r5 = __fdiv_rn(xv, c5.s);
-            const uint32_t a4 = __nv_cvt_float2_to_fp8x2(make_float2(f4, r4), __NV_SATFINITE, __NV_E4M3);
-            const uint32_t a5 = __nv_cvt_float2_to_fp8x2(make_float2(f5, r5), __NV_SATFINITE, __NV_E5M2);
-            bad4 += (a4 & 0xffu) != (a4 >> 8);
-            bad5 += (a5 & 0xffu) != (a5 >> 8);
-        }
-    }
+    const unsigned long long bad4 = selftest_amax<FP8DIT_E4M3FN>(amax_bits);
+    const unsigned long long bad5 = selftest_amax<FP8DIT_E5M2>(amax_bits);
     if (bad4) atomicAdd(&mismatch[0], bad4);
     if (bad5) atomicAdd(&mismatch[1], bad5);
 }
