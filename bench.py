@@ -73,6 +73,26 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest value any rank holds (identity without a process group).
+    Timing only: the FP8 path itself exchanges nothing between ranks."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    if device is None:
+        device = torch.device("cpu") if dist.get_backend() == "gloo" else torch.device("cuda", torch.cuda.current_device())
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, work_per_step: float, steps: int, max_elapsed_ms: float, scale: float = 1e12) -> float:
+    """Units all ranks processed / the slowest rank's time (weak scaling: each
+    rank runs the full per-GPU workload)."""
+    return world * work_per_step * steps / (max_elapsed_ms * 1e-3) / scale
+
+
 class ClockSampler:
     """NVML sampling of SM clock and throttle reasons during the timed region."""
     REASONS = {
@@ -319,11 +339,7 @@ def main():
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     if fp8.device_error(dev) != 0:
         raise RuntimeError("device error during the timed region")
 
@@ -336,7 +352,7 @@ def main():
         k_ms["gemm_down"].append(e[3].elapsed_time(e[4]))
     k_avg = {k: sum(v) / len(v) for k, v in k_ms.items()}
 
-    value = world * FLOPS_PER_STEP * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = whole_job_rate(world, FLOPS_PER_STEP, args.steps, elapsed_ms)
     peaks, peak_src = load_peaks()
     region_s = elapsed_ms * 1e-3
     sustained = region_s > 2.0
@@ -419,12 +435,8 @@ def measure_e2e(fp8, torch, layers, host, dev, args, world):
         step()
     t1.record(stream)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": world * FLOPS_PER_STEP * steps / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
+    return {"value": whole_job_rate(world, FLOPS_PER_STEP, steps, ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "api": "FP8Linear.forward (fp8_scaled_linear) + pinned host copies"}
 
