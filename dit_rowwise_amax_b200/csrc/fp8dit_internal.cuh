@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/fp8dit.h"
 
 namespace fp8dit {
@@ -106,6 +108,35 @@ constexpr int kGemmStoreBox = 32;
 cudaError_t launch_gemm(int cfg, const GemmArgs& args, int units, cudaStream_t stream);
 int gemm_units_for(int cfg, int num_tiles, const DeviceInfo* dev);
 
+// Launch `kernel` on `stream` with programmatic stream serialisation allowed
+// (and a cluster of `cluster_x` CTAs when > 1).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       int cluster_x, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------ device side
 #if defined(__CUDACC__)
 
@@ -183,6 +214,15 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
+
+// ---- programmatic dependent launch: a kernel launched with the PDL attribute
+// may start while its predecessor in the stream finishes; it must not touch
+// global memory the predecessor may write or read before pdl_wait() returns
+// (which waits for the predecessor's completion and memory flush).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the successor in the stream start launching (its own pdl_wait still
+// waits for this kernel to complete).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---- clusters (2-CTA MMA pairs)
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -147,6 +147,10 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     bool aborted = false;
+    // The prologue above touched no global memory; from here on A, W, the
+    // scales and y may belong to the previous kernel in the stream.
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -408,21 +412,8 @@ cudaError_t launch_cfg(const GemmArgs& args, int units, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(units * CG), 1, 1);
-    cfg.blockDim = dim3(C::THREADS, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = CG;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gemm_e4m3_kernel<CG, BN>, args);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return launch_pdl(gemm_e4m3_kernel<CG, BN>, dim3((unsigned)(units * CG)), dim3(C::THREADS), C::SMEM_BYTES,
+                      stream, CG, args);
 }
 
 }  // namespace

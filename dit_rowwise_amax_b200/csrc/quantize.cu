@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* _
 
     uint4 cur[VPT], nxt[VPT];
     int64_t g = blockIdx.x;
+    pdl_wait();  // x may be the previous kernel's output; q and scale its input
+    pdl_trigger();
     load_group<TPR, VPT>(x, M, nvec, ldx, g, cur);
     for (int it = 0; g < groups; g += gridDim.x, ++it) {
         const int64_t gn = g + gridDim.x;
@@ -112,6 +114,8 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_
                                                                      float* __restrict__ scale) {
     __shared__ uint32_t red[kThreads / 32];
     const int64_t nvec = K >> 3;
+    pdl_wait();
+    pdl_trigger();
     for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
         const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
         uint32_t packed = 0;
@@ -152,9 +156,8 @@ cudaError_t launch_regs(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, ui
     }
     const int64_t groups = (M + RPB - 1) / RPB;
     const int64_t grid = std::min<int64_t>(groups, (int64_t)dev->num_sms * per_sm);
-    quantize_rows_regs<TPR, VPT, FMT><<<(unsigned)grid, kThreads, 0, stream>>>(x, M, (int32_t)K, ldx, q, ldq,
-                                                                                scale, groups);
-    return cudaGetLastError();
+    return launch_pdl(quantize_rows_regs<TPR, VPT, FMT>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, x, M,
+                      (int32_t)K, ldx, q, ldq, scale, groups);
 }
 
 template <int FMT>
@@ -163,8 +166,8 @@ cudaError_t launch_fmt(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uin
     const int64_t nvec = K / 8;
     if (nvec > 1024) {
         const int64_t grid = std::min<int64_t>(M, (int64_t)dev->num_sms * 8);
-        quantize_rows_two_pass<FMT><<<(unsigned)grid, kThreads, 0, stream>>>(x, M, K, ldx, q, ldq, scale);
-        return cudaGetLastError();
+        return launch_pdl(quantize_rows_two_pass<FMT>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, x, M, K,
+                          ldx, q, ldq, scale);
     }
     // Smallest power-of-two group (>= 8 threads) that covers the row with <= 4 vectors each.
     int tpr = 8;
