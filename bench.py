@@ -499,6 +499,49 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
             qb = 3 * M * 2048 + 4 * M
             out["quantizer_hidden"] = {"us": qms * 1e3, "gbs": qb / (qms * 1e-3) / 1e9,
                                        "frac_of_hbm": qb / (qms * 1e-3) / 1e9 / hbm_peak}
+    # Merged Q/K/V projection (one N = 6144 GEMM) vs the three separate,
+    # grouped projections above, on hidden_states (HunyuanVideo page §三.4).
+    A = [up(att["hidden"]) for _ in range(2)]
+    M = att["hidden"].shape[0]
+    w_qkv = np.concatenate([att["W_q"], att["W_k"], att["W_v"]], axis=0)
+    b_qkv = np.concatenate([att["bias_q"], att["bias_k"], att["bias_v"]], axis=0)
+    merged = fp8.FP8Linear.from_weight(up(w_qkv), up(b_qkv))
+    qa = torch.empty((M, 2048), dtype=torch.uint8, device=dev)
+    sa = torch.empty((M,), dtype=torch.float32, device=dev)
+    ym = [torch.empty((M, 6144), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    ms = time_region(torch, lambda i: merged.forward(A[i % 2], y=ym[i % 2], qa_scratch=qa, sa_scratch=sa), 50, dev)
+    flops = 2.0 * M * 6144 * 2048
+    out["attention_qkv_merged_n6144"] = {"M": M, "us": ms * 1e3, "tflops": flops / (ms * 1e-3) / 1e12}
+    del A, ym
+
+    # Producer fusion (HunyuanVideo page §三.5): FFN-down fed by GELU(h), h the
+    # FFN-up output. Fused: one kernel emits (FP8, scale). Unfused: torch's
+    # bf16 GELU, then the rowwise quantiser. Both then run the FFN-down GEMM.
+    du, dd = synth.ffn_up(), synth.ffn_down()
+    lu = fp8.FP8Linear.from_weight(up(du["W"]), up(du["bias"]))
+    ld = fp8.FP8Linear.from_weight(up(dd["W"]), up(dd["bias"]))
+    hs = [lu.forward(up(du["A"])) for _ in range(2)]  # [4096, 8192] bf16
+    qd = torch.empty((4096, 8192), dtype=torch.uint8, device=dev)
+    sd = torch.empty((4096,), dtype=torch.float32, device=dev)
+    yd = torch.empty((4096, 2048), dtype=torch.bfloat16, device=dev)
+
+    def fused(i):
+        fp8.act_quantize_rowwise(hs[i % 2], "gelu", q=qd, scale=sd)
+        ld.forward_fp8(qd, sd, y=yd)
+
+    def unfused(i):
+        g = torch.nn.functional.gelu(hs[i % 2])
+        fp8.quantize_rowwise(g, q=qd, scale=sd)
+        ld.forward_fp8(qd, sd, y=yd)
+
+    f_ms = time_region(torch, fused, 50, dev)
+    u_ms = time_region(torch, unfused, 50, dev)
+    a_ms = time_region(torch, lambda i: fp8.act_quantize_rowwise(hs[i % 2], "gelu", q=qd, scale=sd), 50, dev)
+    out["producer_fusion_ffn_down"] = {"fused_us": f_ms * 1e3, "unfused_torch_gelu_us": u_ms * 1e3,
+                                       "gelu_quantize_us": a_ms * 1e3,
+                                       "gelu_quantize_gbs": 3 * 4096 * 8192 / (a_ms * 1e-3) / 1e9}
+    del hs
+
     # GEMM only (pre-quantised activations) at the FFN shapes.
     for name, M, N, K in FFN:
         d = synth.ffn_up() if name == "up" else synth.ffn_down()

@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "E4M3FN", "E5M2", "Fp8DitError", "FP8Linear", "library_path", "load_library",
-    "quantize_rowwise", "quantize_weight_per_channel", "quantize_per_tensor", "convert_state_dict",
+    "quantize_rowwise", "act_quantize_rowwise", "quantize_weight_per_channel", "quantize_per_tensor", "convert_state_dict",
     "scaled_linear_multi", "device_error", "selftest_expired_wait", "selftest_quotient", "as_float8",
 ]
 
@@ -65,6 +65,7 @@ def load_library():
     p, i64, i32, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
     L.fp8_quantize_rowwise.argtypes = [p, i64, i64, i64, ctypes.c_int, p, i64, p, p]
     L.fp8_quantize_weight_per_channel.argtypes = [p, i64, i64, ctypes.c_int, p, p, p]
+    L.fp8_act_quantize_rowwise.argtypes = [p, i64, i64, i64, ctypes.c_int, p, i64, p, p, i64, p]
     L.fp8_quantize_weight_per_tensor_workspace_size.argtypes = [i32]
     L.fp8_quantize_weight_per_tensor_workspace_size.restype = ctypes.c_size_t
     L.fp8_quantize_weight_per_tensor.argtypes = [ctypes.POINTER(_TensorDesc), i32, ctypes.c_int, p,
@@ -79,7 +80,8 @@ def load_library():
     L.fp8dit_selftest_expired_wait.argtypes = [i64, p]
     L.fp8dit_selftest_quotient.argtypes = [p, p]
     L.fp8dit_last_error_string.restype = ctypes.c_char_p
-    for name in ("fp8_quantize_rowwise", "fp8_quantize_weight_per_channel", "fp8_quantize_weight_per_tensor",
+    for name in ("fp8_quantize_rowwise", "fp8_act_quantize_rowwise", "fp8_quantize_weight_per_channel",
+                 "fp8_quantize_weight_per_tensor",
                  "fp8_linear_create", "fp8_linear_destroy", "fp8_scaled_linear", "fp8_scaled_linear_multi",
                  "fp8_scaled_linear_noalloc",
                  "fp8_linear_plan", "fp8dit_device_error", "fp8dit_selftest_expired_wait",
@@ -133,6 +135,30 @@ def quantize_rowwise(x: torch.Tensor, fmt=E4M3FN, q: Optional[torch.Tensor] = No
     _check(load_library().fp8_quantize_rowwise(x.data_ptr(), M, K, x.stride(0), _fmt(fmt), q.data_ptr(),
                                                q.stride(0), scale.data_ptr(), _stream(x.device)))
     return q, scale
+
+
+ACTIVATIONS = {"gelu": 1, "gelu_erf": 1, "gelu_tanh": 2, "silu": 3}
+
+
+def act_quantize_rowwise(h: torch.Tensor, act: str = "gelu", q: Optional[torch.Tensor] = None,
+                         scale: Optional[torch.Tensor] = None, return_bf16: bool = False):
+    """Producer fusion: bf16(act(h)) quantised per token to E4M3FN in one pass.
+    Returns (codes uint8 [M, K], S float32 [M]) and, with return_bf16, the bf16 activation."""
+    h = _bf16_matrix(h, "h")
+    M, K = h.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=h.device)
+    if scale is None:
+        scale = torch.empty((M,), dtype=torch.float32, device=h.device)
+    g = torch.empty((M, K), dtype=torch.bfloat16, device=h.device) if return_bf16 else None
+    try:
+        kind = ACTIVATIONS[act]
+    except KeyError:
+        raise ValueError(f"unknown activation {act!r}") from None
+    _check(load_library().fp8_act_quantize_rowwise(h.data_ptr(), M, K, h.stride(0), kind, q.data_ptr(), q.stride(0),
+                                                   scale.data_ptr(), None if g is None else g.data_ptr(),
+                                                   K if g is not None else 0, _stream(h.device)))
+    return (q, scale, g) if return_bf16 else (q, scale)
 
 
 def quantize_weight_per_channel(w: torch.Tensor, fmt=E4M3FN) -> Tuple[torch.Tensor, torch.Tensor]:

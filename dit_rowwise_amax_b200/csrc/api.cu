@@ -246,6 +246,28 @@ fp8dit_status fp8_quantize_rowwise(const uint16_t* x, int64_t M, int64_t K, int6
     return e == cudaSuccess ? FP8DIT_OK : cuda_fail(e, "rowwise quantise launch");
 }
 
+fp8dit_status fp8_act_quantize_rowwise(const uint16_t* h, int64_t M, int64_t K, int64_t ldh,
+                                       fp8dit_activation act, uint8_t* q, int64_t ldq, float* scale,
+                                       uint16_t* gout, int64_t ldg, fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (act != FP8DIT_ACT_GELU_ERF && act != FP8DIT_ACT_GELU_TANH && act != FP8DIT_ACT_SILU)
+        return invalid("activation");
+    if (M < 0 || K <= 0) return invalid("M must be >= 0 and K > 0");
+    if (K % 16 != 0) return unsupported("K must be a multiple of 16");
+    if (ldh < K || ldh % 8 != 0) return invalid("ldh must be >= K and a multiple of 8");
+    if (ldq < K || ldq % 16 != 0) return invalid("ldq must be >= K and a multiple of 16");
+    if (gout && (ldg < K || ldg % 8 != 0)) return invalid("ldg must be >= K and a multiple of 8");
+    if (M > kMaxRows || K > kMaxK) return unsupported("M or K too large");
+    if (M == 0) return FP8DIT_OK;
+    if (!h || !q || !scale) return invalid("null pointer");
+    if (!aligned16(h) || !aligned16(q) || (gout && !aligned16(gout))) return invalid("h, q and gout must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(scale) & 3u) return invalid("scale must be 4-byte aligned");
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    cudaError_t e = launch_act_quantize_rows(h, M, K, ldh, act, q, ldq, scale, gout, ldg, (cudaStream_t)stream, dev);
+    return e == cudaSuccess ? FP8DIT_OK : cuda_fail(e, "activation quantise launch");
+}
+
 fp8dit_status fp8_quantize_weight_per_channel(const uint16_t* w, int64_t N, int64_t K, fp8dit_format fmt,
                                               uint8_t* qw, float* sw, fp8dit_stream_t stream) {
     t_last_error[0] = 0;

@@ -53,6 +53,9 @@ fp8dit_status encode_tma_2d(CUtensorMap* map, int elem_bytes, const void* base, 
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int fmt,
                                  uint8_t* q, int64_t ldq, float* scale, cudaStream_t stream,
                                  const DeviceInfo* dev);
+cudaError_t launch_act_quantize_rows(const uint16_t* h, int64_t M, int64_t K, int64_t ldh, int act, uint8_t* q,
+                                     int64_t ldq, float* scale, uint16_t* g, int64_t ldg, cudaStream_t stream,
+                                     const DeviceInfo* dev);
 
 struct PerTensorDevDesc {
     const uint16_t* src;

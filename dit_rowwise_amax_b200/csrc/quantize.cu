@@ -17,7 +17,17 @@
 // current one, so HBM reads overlap the arithmetic. Rows longer than
 // 256 threads x 4 vectors x 8 = 8192 elements take a two-pass kernel whose
 // second read of the row comes from L2.
+//
+// Producer fusion ("从 BF16 到 FP8", section 三.5): with ACT != 0 the kernels
+// first replace each loaded element by bf16(act(x)) — GELU (erf or tanh form)
+// or SiLU, evaluated in fp32 with erfcf / expf in forms that do not cancel
+// for negative x — optionally store that bf16 tensor, and quantise it.
+// A bf16 input has only 65536 values, so bf16(act(x)) is evaluated once per
+// device for every bf16 pattern into a 128 KB table (act_table_kernel) and the
+// quantisers read the table: the same values, one cached load per element
+// instead of an erfc / exp evaluation.
 #include <algorithm>
+#include <mutex>
 
 #include "fp8_codec.cuh"
 
@@ -25,6 +35,53 @@ namespace fp8dit {
 namespace {
 
 constexpr int kThreads = 256;
+
+// x / (1 + exp(-t)) without overflow: for t < 0 it is x e^t / (1 + e^t).
+__device__ __forceinline__ float x_logistic(float x, float t) {
+    if (t >= 0.0f) return x / (1.0f + expf(-t));
+    const float e = expf(t);
+    return (x * e) / (1.0f + e);
+}
+
+template <int ACT>
+__device__ __forceinline__ float act_f(float x) {
+    if constexpr (ACT == FP8DIT_ACT_GELU_ERF) {
+        return 0.5f * x * erfcf(-x * 0.70710678118654752f);  // x Phi(x)
+    } else if constexpr (ACT == FP8DIT_ACT_GELU_TANH) {
+        const float u = 0.79788456080286536f * (x + 0.044715f * x * x * x);
+        return x_logistic(x, 2.0f * u);  // x/2 (1 + tanh u)
+    } else if constexpr (ACT == FP8DIT_ACT_SILU) {
+        return x_logistic(x, x);
+    } else {
+        return x;
+    }
+}
+
+// bf16(act(x)) for every bf16 pattern x, one table per activation.
+__device__ uint16_t g_act_table[3][65536];
+
+template <int ACT>
+__global__ void act_table_kernel() {
+    const uint32_t b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= 65536u) return;
+    const __nv_bfloat16 r = __float2bfloat16_rn(act_f<ACT>(__uint_as_float(b << 16)));
+    g_act_table[ACT - 1][b] = *reinterpret_cast<const uint16_t*>(&r);
+}
+
+// bf16(act(x)) for the eight bf16 of a 16-byte vector.
+template <int ACT>
+__device__ __forceinline__ uint4 act8(const uint4& v) {
+    if constexpr (ACT == 0) {
+        return v;
+    } else {
+        const uint16_t* tbl = g_act_table[ACT - 1];
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = (uint32_t)__ldg(tbl + (w[k] & 0xffffu)) | ((uint32_t)__ldg(tbl + (w[k] >> 16)) << 16);
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
 
 template <int TPR, int VPT>
 __device__ __forceinline__ void load_group(const uint16_t* __restrict__ x, int64_t M, int nvec, int64_t ldx,
@@ -42,11 +99,12 @@ __device__ __forceinline__ void load_group(const uint16_t* __restrict__ x, int64
 }
 
 // TPR threads per row (power of two, 8..256), VPT 16-byte vectors per thread.
-template <int TPR, int VPT, int FMT>
+template <int TPR, int VPT, int FMT, int ACT>
 __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* __restrict__ x, int64_t M,
                                                                  int32_t K, int64_t ldx, uint8_t* __restrict__ q,
                                                                  int64_t ldq, float* __restrict__ scale,
-                                                                 int64_t groups) {
+                                                                 int64_t groups, uint16_t* __restrict__ gout,
+                                                                 int64_t ldg) {
     constexpr int RPB = kThreads / TPR;
     constexpr int WPR = TPR / 32;  // warps per row (when TPR >= 32)
     __shared__ uint32_t red[2][kThreads / 32];
@@ -62,6 +120,19 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* _
     for (int it = 0; g < groups; g += gridDim.x, ++it) {
         const int64_t gn = g + gridDim.x;
         if (gn < groups) load_group<TPR, VPT>(x, M, nvec, ldx, gn, nxt);
+        if constexpr (ACT != 0) {
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) cur[i] = act8<ACT>(cur[i]);
+            const int64_t row = g * RPB + r;
+            if (gout != nullptr && row < M) {
+                uint4* gr = reinterpret_cast<uint4*>(gout + row * ldg);
+#pragma unroll
+                for (int i = 0; i < VPT; ++i) {
+                    const int vi = i * TPR + t;
+                    if (vi < nvec) gr[vi] = cur[i];
+                }
+            }
+        }
 
         uint32_t packed = 0;
 #pragma unroll
@@ -107,11 +178,12 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* _
 
 // One block per row (grid-strided): amax pass, then a quantise pass that
 // re-reads the row (from L2). For rows beyond the register-resident kernel.
-template <int FMT>
+template <int FMT, int ACT>
 __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_t* __restrict__ x, int64_t M,
                                                                      int64_t K, int64_t ldx,
                                                                      uint8_t* __restrict__ q, int64_t ldq,
-                                                                     float* __restrict__ scale) {
+                                                                     float* __restrict__ scale,
+                                                                     uint16_t* __restrict__ gout, int64_t ldg) {
     __shared__ uint32_t red[kThreads / 32];
     const int64_t nvec = K >> 3;
     pdl_wait();
@@ -119,7 +191,8 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_
     for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
         const uint4* xr = reinterpret_cast<const uint4*>(x + row * ldx);
         uint32_t packed = 0;
-        for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads) packed = absmax8(__ldg(xr + vi), packed);
+        for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads)
+            packed = absmax8(act8<ACT>(__ldg(xr + vi)), packed);
         uint32_t m = fold_halves(packed);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -132,42 +205,49 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_
         const ScaleCtx c = scale_ctx<FMT>(bf16_bits_to_float(m));
         const Quot2 q2 = quot2_of(c);
         uint8_t* qr = q + row * ldq;
-        if (c.fast) {
-            for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads)
-                *reinterpret_cast<uint2*>(qr + vi * 8) = quant8<FMT, true>(__ldcs(xr + vi), q2);
-        } else {
-            for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads)
-                *reinterpret_cast<uint2*>(qr + vi * 8) = quant8<FMT, false>(__ldcs(xr + vi), q2);
+        uint4* gr = gout != nullptr ? reinterpret_cast<uint4*>(gout + row * ldg) : nullptr;
+        for (int64_t vi = threadIdx.x; vi < nvec; vi += kThreads) {
+            const uint4 v = act8<ACT>(__ldcs(xr + vi));
+            if (ACT != 0 && gr != nullptr) gr[vi] = v;
+            *reinterpret_cast<uint2*>(qr + vi * 8) = c.fast ? quant8<FMT, true>(v, q2) : quant8<FMT, false>(v, q2);
         }
         if (threadIdx.x == 0) scale[row] = c.s;
     }
 }
 
-template <int TPR, int VPT, int FMT>
-cudaError_t launch_regs(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
-                        float* scale, cudaStream_t stream, const DeviceInfo* dev) {
+struct RowsArgs {
+    const uint16_t* x;
+    int64_t M, K, ldx;
+    uint8_t* q;
+    int64_t ldq;
+    float* scale;
+    uint16_t* g;
+    int64_t ldg;
+};
+
+template <int TPR, int VPT, int FMT, int ACT>
+cudaError_t launch_regs(const RowsArgs& a, cudaStream_t stream, const DeviceInfo* dev) {
     constexpr int RPB = kThreads / TPR;
     static int per_sm = 0;  // resident blocks per SM (same on every sm_100a device)
     if (per_sm == 0) {
-        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_rows_regs<TPR, VPT, FMT>,
-                                                                       kThreads, 0);
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &per_sm, quantize_rows_regs<TPR, VPT, FMT, ACT>, kThreads, 0);
         if (e != cudaSuccess) return e;
         if (per_sm < 1) per_sm = 1;
     }
-    const int64_t groups = (M + RPB - 1) / RPB;
+    const int64_t groups = (a.M + RPB - 1) / RPB;
     const int64_t grid = std::min<int64_t>(groups, (int64_t)dev->num_sms * per_sm);
-    return launch_pdl(quantize_rows_regs<TPR, VPT, FMT>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, x, M,
-                      (int32_t)K, ldx, q, ldq, scale, groups);
+    return launch_pdl(quantize_rows_regs<TPR, VPT, FMT, ACT>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1,
+                      a.x, a.M, (int32_t)a.K, a.ldx, a.q, a.ldq, a.scale, groups, a.g, a.ldg);
 }
 
-template <int FMT>
-cudaError_t launch_fmt(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
-                       float* scale, cudaStream_t stream, const DeviceInfo* dev) {
-    const int64_t nvec = K / 8;
+template <int FMT, int ACT>
+cudaError_t launch_fmt(const RowsArgs& a, cudaStream_t stream, const DeviceInfo* dev) {
+    const int64_t nvec = a.K / 8;
     if (nvec > 1024) {
-        const int64_t grid = std::min<int64_t>(M, (int64_t)dev->num_sms * 8);
-        return launch_pdl(quantize_rows_two_pass<FMT>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, x, M, K,
-                          ldx, q, ldq, scale);
+        const int64_t grid = std::min<int64_t>(a.M, (int64_t)dev->num_sms * 8);
+        return launch_pdl(quantize_rows_two_pass<FMT, ACT>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, a.x,
+                          a.M, a.K, a.ldx, a.q, a.ldq, a.scale, a.g, a.ldg);
     }
     // Smallest power-of-two group (>= 8 threads) that covers the row with <= 4 vectors each.
     int tpr = 8;
@@ -175,8 +255,7 @@ cudaError_t launch_fmt(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, uin
     const bool two = nvec <= tpr * 2;
 #define FP8DIT_Q_CASE(T)                                                                        \
     case T:                                                                                     \
-        return two ? launch_regs<T, 2, FMT>(x, M, K, ldx, q, ldq, scale, stream, dev)           \
-                   : launch_regs<T, 4, FMT>(x, M, K, ldx, q, ldq, scale, stream, dev);
+        return two ? launch_regs<T, 2, FMT, ACT>(a, stream, dev) : launch_regs<T, 4, FMT, ACT>(a, stream, dev);
     switch (tpr) {
         FP8DIT_Q_CASE(8)
         FP8DIT_Q_CASE(16)
@@ -225,8 +304,48 @@ __global__ void selftest_quotient_kernel(unsigned long long* mismatch) {
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int fmt, uint8_t* q,
                                  int64_t ldq, float* scale, cudaStream_t stream, const DeviceInfo* dev) {
     if (M == 0) return cudaSuccess;
-    return fmt == FP8DIT_E4M3FN ? launch_fmt<FP8DIT_E4M3FN>(x, M, K, ldx, q, ldq, scale, stream, dev)
-                                : launch_fmt<FP8DIT_E5M2>(x, M, K, ldx, q, ldq, scale, stream, dev);
+    const RowsArgs a{x, M, K, ldx, q, ldq, scale, nullptr, 0};
+    return fmt == FP8DIT_E4M3FN ? launch_fmt<FP8DIT_E4M3FN, 0>(a, stream, dev)
+                                : launch_fmt<FP8DIT_E5M2, 0>(a, stream, dev);
+}
+
+// Builds the activation tables on the current device once (on `stream`, which
+// is then synchronised, so later calls on any stream see the tables).
+static cudaError_t ensure_act_tables(cudaStream_t stream) {
+    static std::mutex mu;
+    static bool ready[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (ready[dev]) return cudaSuccess;
+    act_table_kernel<FP8DIT_ACT_GELU_ERF><<<256, 256, 0, stream>>>();
+    act_table_kernel<FP8DIT_ACT_GELU_TANH><<<256, 256, 0, stream>>>();
+    act_table_kernel<FP8DIT_ACT_SILU><<<256, 256, 0, stream>>>();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaStreamSynchronize(stream)) != cudaSuccess) return e;
+    ready[dev] = true;
+    return cudaSuccess;
+}
+
+cudaError_t launch_act_quantize_rows(const uint16_t* h, int64_t M, int64_t K, int64_t ldh, int act, uint8_t* q,
+                                     int64_t ldq, float* scale, uint16_t* g, int64_t ldg, cudaStream_t stream,
+                                     const DeviceInfo* dev) {
+    if (M == 0) return cudaSuccess;
+    cudaError_t e = ensure_act_tables(stream);
+    if (e != cudaSuccess) return e;
+    const RowsArgs a{h, M, K, ldh, q, ldq, scale, g, ldg};
+    switch (act) {
+        case FP8DIT_ACT_GELU_ERF:
+            return launch_fmt<FP8DIT_E4M3FN, FP8DIT_ACT_GELU_ERF>(a, stream, dev);
+        case FP8DIT_ACT_GELU_TANH:
+            return launch_fmt<FP8DIT_E4M3FN, FP8DIT_ACT_GELU_TANH>(a, stream, dev);
+        case FP8DIT_ACT_SILU:
+            return launch_fmt<FP8DIT_E4M3FN, FP8DIT_ACT_SILU>(a, stream, dev);
+        default:
+            return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_selftest_quotient(unsigned long long* mismatch, cudaStream_t stream) {

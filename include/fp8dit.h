@@ -81,6 +81,30 @@ fp8dit_status fp8_quantize_rowwise(const uint16_t* x, int64_t M, int64_t K, int6
                                    fp8dit_format fmt, uint8_t* q, int64_t ldq, float* scale,
                                    fp8dit_stream_t stream);
 
+/* Activations a producer kernel can apply before quantising. */
+typedef enum {
+    FP8DIT_ACT_GELU_ERF = 1,  /* x Phi(x) = x/2 (1 + erf(x / sqrt 2)) */
+    FP8DIT_ACT_GELU_TANH = 2, /* x/2 (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) */
+    FP8DIT_ACT_SILU = 3       /* x / (1 + exp(-x)) */
+} fp8dit_activation;
+
+/*
+ * Producer fusion ("从 BF16 到 FP8", section 三.5): the GELU / SiLU in front of
+ * FFN-down emits the (FP8 tensor, per-token scale) pair directly instead of a
+ * bf16 tensor that a separate pass then quantises.
+ *   h     [M, K] bf16 (the FFN-up output), row stride ldh elements (ldh % 8 == 0), 16-byte aligned.
+ *   g     = bf16_rne(act(h)), evaluated in fp32 (CUDA erfcf / expf); stored to
+ *         gout [M, K] (row stride ldg, 16-byte aligned) when gout != NULL.
+ *   q, scale: the rowwise recipe applied to g, E4M3FN codes (the GEMM's input).
+ * Same shape rules as fp8_quantize_rowwise. The first call on a device builds
+ * a 128 KB table per activation (bf16(act(x)) for all 65536 bf16 x, in static
+ * device memory) and synchronises `stream` once; make that first call before
+ * any stream capture.
+ */
+fp8dit_status fp8_act_quantize_rowwise(const uint16_t* h, int64_t M, int64_t K, int64_t ldh,
+                                       fp8dit_activation act, uint8_t* q, int64_t ldq, float* scale,
+                                       uint16_t* gout, int64_t ldg, fp8dit_stream_t stream);
+
 /*
  * Per-output-channel quantisation of a bf16 weight W [N, K] (K contiguous):
  * the rowwise recipe applied to each of the N rows, producing the K-major

@@ -10,6 +10,8 @@ What it computes (see oracle.c for the page citations):
   * ``quantize_tensor``: the same with one amax per tensor.
   * ``linear``: exact integer dot of dequantised E4M3 operands, then
     y = dot * sa[m] * sw[n] + bias[n] in double.
+  * ``act_bf16``: the producer activation (GELU erf / tanh form, SiLU) in
+    double, rounded once to bf16.
 """
 from __future__ import annotations
 
@@ -61,6 +63,12 @@ def _load():
         lib.or_linear.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p]
         lib.or_linear_at.restype = None
         lib.or_linear_at.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _p, _i64, _p]
+        lib.or_act.restype = ctypes.c_double
+        lib.or_act.argtypes = [ctypes.c_int, ctypes.c_double]
+        lib.or_round_bf16.restype = ctypes.c_uint16
+        lib.or_round_bf16.argtypes = [ctypes.c_double]
+        lib.or_act_bf16.restype = None
+        lib.or_act_bf16.argtypes = [ctypes.c_int, _p, _i64, _p]
         lib.or_num_threads.restype = ctypes.c_int
         lib.or_num_threads.argtypes = []
         lib.or_dot_units.restype = None
@@ -145,6 +153,29 @@ def dot_units(qa, qw) -> np.ndarray:
     out = np.empty((M, N), dtype=np.int64)
     _load().or_dot_units(qa.ctypes.data, qw.ctypes.data, M, N, K, out.ctypes.data)
     return out
+
+
+ACT_GELU_ERF = 1
+ACT_GELU_TANH = 2
+ACT_SILU = 3
+
+
+def act(kind: int, x: float) -> float:
+    """The producer activation in double."""
+    return float(_load().or_act(kind, x))
+
+
+def round_bf16(v: float) -> int:
+    """Nearest bf16 bit pattern to a double (ties to even)."""
+    return int(_load().or_round_bf16(v))
+
+
+def act_bf16(kind: int, h: np.ndarray) -> np.ndarray:
+    """bf16(act(h)) elementwise; h and the result are uint16 bf16 patterns."""
+    h = _c(h, np.uint16)
+    g = np.empty(h.shape, dtype=np.uint16)
+    _load().or_act_bf16(kind, h.ctypes.data, h.size, g.ctypes.data)
+    return g
 
 
 def num_threads() -> int:

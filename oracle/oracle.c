@@ -207,6 +207,62 @@ void or_dot_units(const uint8_t* qa, const uint8_t* qw, int64_t M, int64_t N, in
         }
 }
 
+/* ----------------------------------------------------- producer activations */
+/*
+ * "从 BF16 到 FP8：HunyuanVideo1.5推理优化复盘", section 三.5: the GELU / SiLU that
+ * precedes FFN-down emits its output straight to FP8 with a per-token scale.
+ * The activation is evaluated in double and rounded once to bf16; that bf16
+ * tensor is what the rowwise recipe quantises.
+ *   act 1: GELU, erf form   x Phi(x) = x/2 (1 + erf(x / sqrt 2)) = x/2 erfc(-x / sqrt 2)
+ *   act 2: GELU, tanh form  x/2 (1 + tanh(u)) = x / (1 + exp(-2u)),
+ *                           u = sqrt(2/pi) (x + 0.044715 x^3)
+ *   act 3: SiLU             x / (1 + exp(-x))
+ * The right-hand forms are the same functions without the cancellation of
+ * 1 + erf / 1 + tanh for negative x.
+ */
+enum { OR_ACT_GELU_ERF = 1, OR_ACT_GELU_TANH = 2, OR_ACT_SILU = 3 };
+
+double or_act(int act, double x) {
+    switch (act) {
+        case OR_ACT_GELU_ERF:
+            return 0.5 * x * erfc(-x / sqrt(2.0));
+        case OR_ACT_GELU_TANH:
+            return x / (1.0 + exp(-2.0 * sqrt(2.0 / M_PI) * (x + 0.044715 * x * x * x)));
+        case OR_ACT_SILU:
+            return x / (1.0 + exp(-x));
+        default:
+            return x;
+    }
+}
+
+/* Nearest bf16 to a double (ties to even), as a bit pattern; finite inputs
+ * within the bf16 range. One rounding, straight from double. */
+uint16_t or_round_bf16(double v) {
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    int e;
+    if (a < ldexp(1.0, -126)) {
+        e = -126; /* subnormal bf16 spacing */
+    } else {
+        int fe;
+        frexp(a, &fe);
+        e = fe - 1;
+    }
+    double quantum = ldexp(1.0, e - 7);
+    double r = rint(a / quantum) * quantum; /* representable in bf16, hence in fp32 */
+    float f = (float)r;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return sign | (uint16_t)(u >> 16);
+}
+
+/* g[i] = bf16(act(h[i])) for n elements. */
+void or_act_bf16(int act, const uint16_t* h, int64_t n, uint16_t* g) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) g[i] = or_round_bf16(or_act(act, (double)or_bf16_to_f32(h[i])));
+}
+
 /* Encode a batch of fp32 values (for codec tests). */
 void or_encode_many(int fmt, const float* v, int64_t n, uint8_t* out) {
 #pragma omp parallel for schedule(static)

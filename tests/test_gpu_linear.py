@@ -97,6 +97,18 @@ def test_ragged_shapes(M, N, K):
     check_full(y, qa, sa, qw, sw, bias)
 
 
+@pytest.mark.parametrize("M,N,K", [(300, 8, 16), (200, 24, 16384), (513, 264, 4112), (257, 2048, 2048)])
+def test_extreme_shapes(M, N, K):
+    """Smallest N, the longest K (two-pass quantiser, 128 k-blocks), K not a
+    multiple of the 128-wide k-block, and M just past a 256-row pair tile."""
+    A = synth.normal_bf16(f"gpu/ext/A/{M}x{K}", (M, K), 1.0, outlier_p=0.01, outlier_factor=20.0)
+    W = synth.normal_bf16(f"gpu/ext/W/{N}x{K}", (N, K), 0.02)
+    bias = synth.normal_bf16(f"gpu/ext/b/{N}", (N,), 0.1)
+    layer, qw, sw = make_layer(W, bias)
+    y, qa, sa = run_bf16(layer, A)
+    check_full(y, qa, sa, qw, sw, bias)
+
+
 def test_no_bias():
     d = synth.tiny()
     layer, qw, sw = make_layer(d["W"], None)
