@@ -552,6 +552,14 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
         tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
         out[f"gemm_only_ffn_{name}"] = {"us": ms * 1e3, "tflops": tf, "frac_of_fp8_peak": tf / fp8_peak,
                                         "plan": list(layer.plan(M))}
+        # FP8 weight-only (bf16 activation, E4M3 weight decoded in shared
+        # memory, BF16 tensor cores), same layer.
+        a16s = [up(d["A"]) for _ in range(3)]
+        wms = time_region(torch, lambda i: layer.forward_weight_only(a16s[i % 3], y=ys[i % 3]), 100, dev)
+        wtf = 2.0 * M * N * K / (wms * 1e-3) / 1e12
+        out[f"weight_only_ffn_{name}"] = {"us": wms * 1e3, "tflops": wtf,
+                                          "frac_of_bf16_peak": wtf / peaks["bf16_tflops"]}
+        del a16s
         # BF16 context: the same shape through torch.matmul (cuBLAS), bench script only.
         a16 = up(d["A"])
         w16 = up(d["W"])

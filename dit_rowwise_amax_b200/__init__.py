@@ -75,6 +75,7 @@ def load_library():
     L.fp8_scaled_linear.argtypes = [p, i64, p, p, p, p, p, p, p]
     L.fp8_scaled_linear_multi.argtypes = [ctypes.POINTER(p), i32, i64, p, p, p, ctypes.POINTER(p), p]
     L.fp8_scaled_linear_noalloc.argtypes = [p, i64, p, p, p]
+    L.fp8_weight_only_linear.argtypes = [p, i64, p, p, p]
     L.fp8_linear_plan.argtypes = [p, i64, i32, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.fp8dit_device_error.argtypes = [p]
     L.fp8dit_selftest_expired_wait.argtypes = [i64, p]
@@ -83,7 +84,7 @@ def load_library():
     for name in ("fp8_quantize_rowwise", "fp8_act_quantize_rowwise", "fp8_quantize_weight_per_channel",
                  "fp8_quantize_weight_per_tensor",
                  "fp8_linear_create", "fp8_linear_destroy", "fp8_scaled_linear", "fp8_scaled_linear_multi",
-                 "fp8_scaled_linear_noalloc",
+                 "fp8_scaled_linear_noalloc", "fp8_weight_only_linear",
                  "fp8_linear_plan", "fp8dit_device_error", "fp8dit_selftest_expired_wait",
                  "fp8dit_selftest_quotient"):
         getattr(L, name).restype = st
@@ -303,6 +304,18 @@ class FP8Linear:
         return y
 
     __call__ = forward
+
+    def forward_weight_only(self, a: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """FP8 weight-only: bf16 activation (not quantised) x this layer's E4M3
+        weight decoded to bf16, on the BF16 tensor cores."""
+        a = _bf16_matrix(a, "a")
+        if not a.is_contiguous() or a.shape[1] != self.K:
+            raise ValueError(f"a must be contiguous [M, {self.K}]")
+        M = a.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.bfloat16, device=a.device)
+        _check(load_library().fp8_weight_only_linear(self._h, M, a.data_ptr(), y.data_ptr(), _stream(a.device)))
+        return y
 
     def forward_fp8(self, qa: torch.Tensor, sa: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
         if qa.dtype not in (torch.uint8, torch.float8_e4m3fn) or qa.dim() != 2 or not qa.is_contiguous():

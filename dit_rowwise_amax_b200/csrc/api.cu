@@ -181,15 +181,29 @@ static int choose_cfg(const fp8dit_linear_s* h, int64_t M, int n_problems) {
     return kCfg128x128;
 }
 
-static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, const uint8_t* qa, const float* sa,
-                              uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev) {
-    const int cfg = choose_cfg(hs[0], M, n);
+// Weight-only plan: 256 x 256 pair tiles when M fills them and they keep half
+// of the pairs busy, else 128 x 128 tiles on single CTAs.
+static int choose_cfg_weight_only(const fp8dit_linear_s* h, int64_t M) {
+    const int pairs = h->num_sms / 2;
+    if (M >= 256 && tiles_for(h, M, 1, kCfgW8Pair256) * 2 >= pairs) return kCfgW8Pair256;
+    return kCfgW8128x128;
+}
+
+// a: FP8 codes [M, K] (qa) for the FP8 x FP8 configurations, bf16 [M, K] for
+// the weight-only ones; sa: per-token scales, or NULL (weight-only).
+static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, const void* a, const float* sa,
+                              uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev, int cfg) {
     const int bm = gemm_block_m(cfg);
     const int bn = gemm_block_n(cfg);
+    const int ke = gemm_k_elems(cfg);
+    const int64_t K = hs[0]->K;
     GemmArgs args;
     memset(&args, 0, sizeof(args));
-    fp8dit_status st = encode_tma_2d(&args.tmA, 1, qa, (uint64_t)hs[0]->K, (uint64_t)M, (uint64_t)hs[0]->K,
-                                     kGemmBlockK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    fp8dit_status st = gemm_weight_only(cfg)
+                           ? encode_tma_2d(&args.tmA, 2, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, (uint32_t)ke,
+                                           128, CU_TENSOR_MAP_SWIZZLE_128B)
+                           : encode_tma_2d(&args.tmA, 1, a, (uint64_t)K, (uint64_t)M, (uint64_t)K, (uint32_t)ke,
+                                           128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FP8DIT_OK) return st;
     const int tiles_m = (int)((M + bm - 1) / bm);
     int tiles = 0;
@@ -212,7 +226,7 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
     args.G = n;
     args.tiles_m = tiles_m;
     args.num_tiles = tiles;
-    args.num_kb = (int32_t)((hs[0]->K + kGemmBlockK - 1) / kGemmBlockK);
+    args.num_kb = (int32_t)((K + ke - 1) / ke);
     args.err = dev_err(dev);
     cudaError_t e = launch_gemm(cfg, args, gemm_units_for(cfg, tiles, dev), stream);
     if (e != cudaSuccess) return cuda_fail(e, "FP8 GEMM launch");
@@ -343,9 +357,14 @@ fp8dit_status fp8_linear_create(int64_t N, int64_t K, const uint8_t* qw, const f
         h->bias = bias;
         h->device = device;
         h->num_sms = dev->num_sms;
-        for (int cfg = 0; cfg < kNumCfgs && st == FP8DIT_OK; ++cfg)
-            st = encode_tma_2d(&h->tmB[cfg], 1, qw, (uint64_t)K, (uint64_t)N, (uint64_t)K, kGemmBlockK,
-                               (uint32_t)gemm_b_box_rows(cfg), CU_TENSOR_MAP_SWIZZLE_128B);
+        for (int cfg = 0; cfg < kNumCfgs && st == FP8DIT_OK; ++cfg) {
+            // FP8 x FP8: 128-byte rows, 128-byte swizzle (MMA-ready). Weight-only:
+            // 64-byte rows of codes, unswizzled, decoded to bf16 in shared memory.
+            const bool wo = gemm_weight_only(cfg);
+            st = encode_tma_2d(&h->tmB[cfg], 1, qw, (uint64_t)K, (uint64_t)N, (uint64_t)K, (uint32_t)gemm_k_elems(cfg),
+                               (uint32_t)gemm_b_box_rows(cfg),
+                               wo ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+        }
     }
     if (device != prev) cudaSetDevice(prev);
     if (st != FP8DIT_OK) {
@@ -400,7 +419,23 @@ fp8dit_status fp8_scaled_linear(fp8dit_linear h, int64_t M, const uint16_t* a_bf
         qa = qa_scratch;
         sa = sa_scratch;
     }
-    return run_gemm(&h, 1, M, qa, sa, &y, (cudaStream_t)stream, dev);
+    return run_gemm(&h, 1, M, qa, sa, &y, (cudaStream_t)stream, dev, choose_cfg(h, M, 1));
+}
+
+fp8dit_status fp8_weight_only_linear(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, uint16_t* y,
+                                     fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (!h) return invalid("null handle");
+    if (M < 0) return invalid("M must be >= 0");
+    if (M > kMaxRows) return unsupported("M too large");
+    if (M == 0) return FP8DIT_OK;
+    if (!a_bf16 || !aligned16(a_bf16)) return invalid("a_bf16 must be non-null and 16-byte aligned");
+    if (!y || !aligned16(y)) return invalid("y must be non-null and 16-byte aligned");
+    fp8dit_status st = check_device(h);
+    if (st != FP8DIT_OK) return st;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    return run_gemm(&h, 1, M, a_bf16, nullptr, &y, (cudaStream_t)stream, dev, choose_cfg_weight_only(h, M));
 }
 
 fp8dit_status fp8_scaled_linear_multi(const fp8dit_linear* hs, int32_t n, int64_t M, const uint16_t* a_bf16,
@@ -427,7 +462,7 @@ fp8dit_status fp8_scaled_linear_multi(const fp8dit_linear* hs, int32_t n, int64_
     cudaError_t e = launch_quantize_rows(a_bf16, M, hs[0]->K, hs[0]->K, FP8DIT_E4M3FN, qa_scratch, hs[0]->K,
                                          sa_scratch, (cudaStream_t)stream, dev);
     if (e != cudaSuccess) return cuda_fail(e, "activation quantise launch");
-    return run_gemm(hs, n, M, qa_scratch, sa_scratch, ys, (cudaStream_t)stream, dev);
+    return run_gemm(hs, n, M, qa_scratch, sa_scratch, ys, (cudaStream_t)stream, dev, choose_cfg(hs[0], M, n));
 }
 
 fp8dit_status fp8_linear_plan(fp8dit_linear h, int64_t M, int32_t n_problems, int32_t* block_m, int32_t* block_n,

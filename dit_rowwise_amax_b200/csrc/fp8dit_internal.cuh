@@ -96,15 +96,19 @@ struct alignas(64) GemmArgs {
 
 // Tile configurations the plan chooses from.
 enum GemmConfig : int32_t {
-    kCfgPair256 = 0,  // 256 x 256 tile on a 2-CTA pair (cta_group::2)
-    kCfg128x256 = 1,  // 128 x 256 tile on one CTA
-    kCfg128x128 = 2,  // 128 x 128 tile on one CTA
-    kNumCfgs = 3,
+    kCfgPair256 = 0,    // FP8 x FP8: 256 x 256 tile on a 2-CTA pair (cta_group::2)
+    kCfg128x256 = 1,    // FP8 x FP8: 128 x 256 tile on one CTA
+    kCfg128x128 = 2,    // FP8 x FP8: 128 x 128 tile on one CTA
+    kCfgW8Pair256 = 3,  // bf16 x FP8 weight (weight-only): 256 x 256 tile on a 2-CTA pair
+    kCfgW8128x128 = 4,  // bf16 x FP8 weight (weight-only): 128 x 128 tile on one CTA
+    kNumCfgs = 5,
 };
 int gemm_block_m(int cfg);
 int gemm_block_n(int cfg);
 int gemm_b_box_rows(int cfg);
 int gemm_cta_group(int cfg);
+bool gemm_weight_only(int cfg);
+int gemm_k_elems(int cfg);  // K elements per pipeline stage
 constexpr int kGemmBlockK = 128;  // bytes = FP8 elements per k-block (one 128 B swizzle row)
 constexpr int kGemmStoreBox = 32;
 
@@ -305,6 +309,17 @@ __device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32 (kind::f16).
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on `bar` in every CTA of `cta_mask` when this thread's prior pair MMAs complete.
 __device__ __forceinline__ void mma_commit_pair_multicast(uint64_t* bar, uint16_t cta_mask) {
     asm volatile(
@@ -344,6 +359,17 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uin
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32 (kind::f16), one CTA.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -395,6 +421,12 @@ __device__ __forceinline__ uint64_t umma_desc_kmajor_sw128(uint32_t smem_addr) {
 // A / B major 15 / 16 (0 = K), N >> 3 in 17-22, M >> 4 in 24-28.
 __host__ __device__ constexpr uint32_t umma_idesc_e4m3_f32(int M, int N) {
     return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor of kind::f16 with BF16 A and B (format 1 in bits 7-9
+// and 10-12), F32 accumulator, both K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 #endif  // __CUDACC__

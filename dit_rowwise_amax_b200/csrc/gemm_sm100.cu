@@ -34,36 +34,42 @@
 // raises the device error word and its own and its peer's abort flags, lets
 // in-flight copies and MMAs land, frees TMEM and returns.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "fp8dit_internal.cuh"
 
 namespace fp8dit {
 namespace {
 
-template <int CG, int BN>
+template <int CG, int BN, bool W8>
 struct Cfg {
-    static constexpr int BM = 128 * CG;    // rows of one MMA tile
-    static constexpr int ROWS = 128;       // rows per CTA (TMEM lanes)
-    static constexpr int BK = kGemmBlockK;  // 128 FP8 = one 128-byte swizzle row
+    static constexpr int BM = 128 * CG;     // rows of one MMA tile
+    static constexpr int ROWS = 128;        // rows per CTA (TMEM lanes)
+    static constexpr int ROW_BYTES = 128;   // one 128-byte swizzle row per operand row per stage
+    static constexpr int KE = W8 ? 64 : 128;  // K elements per stage (bf16 : FP8)
     static constexpr int B_ROWS = BN / CG;  // W rows per CTA per stage
-    static constexpr int A_BYTES = ROWS * BK;
-    static constexpr int B_BYTES = B_ROWS * BK;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6);
+    static constexpr int A_BYTES = ROWS * ROW_BYTES;
+    static constexpr int B_BYTES = B_ROWS * ROW_BYTES;         // MMA-ready B: FP8, or bf16 decoded from FP8
+    static constexpr int RAW_BYTES = W8 ? B_ROWS * 64 : 0;      // FP8 weight codes as loaded (W8 only)
+    static constexpr int TX_BYTES = A_BYTES + (W8 ? RAW_BYTES : B_BYTES);  // TMA bytes per CTA per stage
+    static constexpr int STAGE_SMEM = A_BYTES + B_BYTES + RAW_BYTES;
+    static constexpr int STAGES = W8 ? (B_ROWS == 256 ? 3 : 5) : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6));
     static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
-    static constexpr int EPI_WARPS = 8;              // two per TMEM lane quarter, each half the columns
-    static constexpr int EPI_COLS = BN / 2;          // columns per epilogue warp
+    static constexpr int EPI_WARPS = W8 ? 4 : 8;     // one or two per TMEM lane quarter
+    static constexpr int CONV_WARPS = W8 ? 4 : 0;    // FP8 -> bf16 weight decoders (W8)
+    static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
     static constexpr int BOX = 32;                   // epilogue store box: 32 rows x 32 columns
     static constexpr int STG_BYTES = BOX * BOX * 2;  // 2 KB, 64-byte rows, one per epilogue warp
     static constexpr int STAGING_BYTES = EPI_WARPS * STG_BYTES;
     static constexpr int SWB_FLOATS = 2 * EPI_COLS;  // sw then bias as fp32, one copy per epilogue warp
     static constexpr int SWB_BYTES = EPI_WARPS * SWB_FLOATS * 4;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
-    static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_SMEM + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
+    static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-    static_assert((2 * STAGES + 2 * ACC + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
+    static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -85,18 +91,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int CG, int BN>
-__global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(const __grid_constant__ GemmArgs args) {
-    using C = Cfg<CG, BN>;
+template <int CG, int BN, bool W8>
+__global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
+    gemm_e4m3_kernel(const __grid_constant__ GemmArgs args) {
+    using C = Cfg<CG, BN, W8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + C::STAGES * C::A_BYTES;
-    uint8_t* staging = sB + C::STAGES * C::B_BYTES;
+    uint8_t* sRaw = sB + C::STAGES * C::B_BYTES;
+    uint8_t* staging = sRaw + C::STAGES * C::RAW_BYTES;
     float* swb = reinterpret_cast<float*>(staging + C::STAGING_BYTES);
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(swb) + C::SWB_BYTES);
     uint64_t* empty = full + C::STAGES;
-    uint64_t* tfull = empty + C::STAGES;
+    uint64_t* conv = empty + C::STAGES;  // W8: decoded B stage ready (arrivals from both CTAs' decoders)
+    uint64_t* tfull = conv + C::STAGES;
     uint64_t* tempty = tfull + C::ACC;
     uint64_t* drain = tempty + C::ACC;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -118,6 +127,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&conv[s], C::CONV_WARPS * CG > 0 ? C::CONV_WARPS * CG : 1);
         }
         for (int a = 0; a < C::ACC; ++a) {
             mbar_init(&tfull[a], 1);
@@ -167,15 +177,21 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
                         abort_peer();
                         break;
                     }
-                    if (CG == 2) {
+                    if (W8) {
+                        // Each CTA tracks its own bf16 A and FP8 W loads; its
+                        // decoder warps wait on them.
+                        mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                        tma_load_2d(sA + stage * C::A_BYTES, &args.tmA, &full[stage], kb * C::KE, a_row);
+                        tma_load_2d(sRaw + stage * C::RAW_BYTES, &args.tmB[tc.g], &full[stage], kb * C::KE, b_row);
+                    } else if (CG == 2) {
                         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
-                        if (leader) mbar_arrive_expect_tx(&full[stage], CG * C::STAGE_BYTES);
-                        tma_load_2d_pair(sA + stage * C::A_BYTES, &args.tmA, bar, kb * C::BK, a_row);
-                        tma_load_2d_pair(sB + stage * C::B_BYTES, &args.tmB[tc.g], bar, kb * C::BK, b_row);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], CG * C::TX_BYTES);
+                        tma_load_2d_pair(sA + stage * C::A_BYTES, &args.tmA, bar, kb * C::KE, a_row);
+                        tma_load_2d_pair(sB + stage * C::B_BYTES, &args.tmB[tc.g], bar, kb * C::KE, b_row);
                     } else {
-                        mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-                        tma_load_2d(sA + stage * C::A_BYTES, &args.tmA, &full[stage], kb * C::BK, a_row);
-                        tma_load_2d(sB + stage * C::B_BYTES, &args.tmB[tc.g], &full[stage], kb * C::BK, b_row);
+                        mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                        tma_load_2d(sA + stage * C::A_BYTES, &args.tmA, &full[stage], kb * C::KE, a_row);
+                        tma_load_2d(sB + stage * C::B_BYTES, &args.tmB[tc.g], &full[stage], kb * C::KE, b_row);
                     }
                     ++armed;
                     if (++stage == C::STAGES) {
@@ -184,7 +200,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
                     }
                 }
             }
-            if (aborted && leader) {
+            if (aborted && (leader || W8)) {
                 // Let every copy signalled on this CTA's barriers land before exit.
                 for (int s = 0; s < C::STAGES; ++s) {
                     if (armed <= s) break;
@@ -197,7 +213,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (pair leader)
         if (lane == 0 && leader) {
-            constexpr uint32_t idesc = umma_idesc_e4m3_f32(C::BM, BN);
+            constexpr uint32_t idesc = W8 ? umma_idesc_bf16_f32(C::BM, BN) : umma_idesc_e4m3_f32(C::BM, BN);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
             for (int t = unit; t < args.num_tiles && !aborted; t += units) {
                 if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, args.err)) {
@@ -208,7 +224,9 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 for (int kb = 0; kb < args.num_kb; ++kb) {
-                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, args.err)) {
+                    // W8: the decoded B of both CTAs (and, through the decoders'
+                    // waits, both CTAs' A) is ready. FP8: both CTAs' TMA loads landed.
+                    if (!mbar_wait_bounded(W8 ? &conv[stage] : &full[stage], phase, abort_flag, args.err)) {
                         aborted = true;
                         abort_peer();
                         break;
@@ -217,11 +235,16 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
                     const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
                     const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-                    for (int j = 0; j < C::BK / 32; ++j) {
+                    for (int j = 0; j < C::ROW_BYTES / 32; ++j) {  // 32 bytes of K per MMA
                         const uint64_t ad = umma_desc_kmajor_sw128(a0 + 32 * j);
                         const uint64_t bd = umma_desc_kmajor_sw128(b0 + 32 * j);
-                        if (CG == 2) mma_f8f6f4_pair(d_tmem, ad, bd, idesc, (kb | j) != 0);
-                        else mma_f8f6f4(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                        if (W8) {
+                            if (CG == 2) mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                            else mma_bf16(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                        } else {
+                            if (CG == 2) mma_f8f6f4_pair(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                            else mma_f8f6f4(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                        }
                     }
                     // The ring slot is free (in both CTAs) once these MMAs have read it.
                     if (CG == 2) mma_commit_pair_multicast(&empty[stage], 0x3);
@@ -245,7 +268,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
             mbar_wait_bounded(drain, 0, nullptr, args.err);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 2 + C::EPI_WARPS) {
         // ------------------------------------------------ epilogue warps
         const int q = warp & 3;          // TMEM lane quarter this warp may access
         const int ew = warp - 2;         // 0..7
@@ -284,7 +307,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
                              : make_uint4(0, 0, 0, 0);
             }
             const int row = tc.tm * C::BM + (int)rank * C::ROWS + q * 32 + lane;
-            p.sa = row < args.M ? __ldg(args.sa + row) : 0.0f;
+            p.sa = row < args.M ? (args.sa != nullptr ? __ldg(args.sa + row) : 1.0f) : 0.0f;
         };
         auto publish = [&](const Pre& p) {  // this warp's smem copy of sw / bias (fp32)
 #pragma unroll
@@ -380,6 +403,59 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
         }
         if (lane == 0) bulk_wait_group<0>();  // all output stores complete
         __syncwarp();
+    } else {
+        // ------------------------------------------------ FP8 -> bf16 weight decoders (W8)
+        // Stage s: sRaw holds B_ROWS rows x 64 FP8 codes (64-byte rows, as
+        // loaded); write them as B_ROWS rows x 64 bf16 (128-byte rows, 128-byte
+        // swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)), the
+        // K-major layout the MMA descriptors describe. E4M3 values are exact
+        // in bf16. Then release the stage to the pair leader's MMA.
+        if constexpr (W8) {
+            const int ct = threadIdx.x - 32 * (2 + C::EPI_WARPS);
+            uint32_t stage = 0, phase = 0;
+            bool stop = false;
+            for (int t = unit; t < args.num_tiles && !stop; t += units) {
+                for (int kb = 0; kb < args.num_kb; ++kb) {
+                    const bool ok = mbar_wait_bounded(&full[stage], phase, abort_flag, args.err);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        if (lane == 0) abort_peer();
+                        stop = true;
+                        break;
+                    }
+                    const uint8_t* raw = sRaw + stage * C::RAW_BYTES;
+                    uint8_t* dst = sB + stage * C::B_BYTES;
+#pragma unroll 2
+                    for (int idx = ct; idx < C::B_ROWS * 4; idx += 32 * C::CONV_WARPS) {
+                        const int r = idx >> 2, c = idx & 3;
+                        const uint4 v = *reinterpret_cast<const uint4*>(raw + r * 64 + c * 16);
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                        uint32_t o[8];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] & 0xffffu), __NV_E4M3);
+                            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> 16), __NV_E4M3);
+                            o[2 * k] = pack_bf16x2(__half2float(__ushort_as_half(lo.x)), __half2float(__ushort_as_half(lo.y)));
+                            o[2 * k + 1] = pack_bf16x2(__half2float(__ushort_as_half(hi.x)), __half2float(__ushort_as_half(hi.y)));
+                        }
+                        *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c) ^ (r & 7)) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4)) =
+                            make_uint4(o[4], o[5], o[6], o[7]);
+                    }
+                    fence_proxy_async_smem();  // the tensor core reads these bytes through the async proxy
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&conv[stage]), 0));
+                        else mbar_arrive(&conv[stage]);
+                    }
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
+        __syncwarp();
     }
 
     if (*abort_flag) {
@@ -399,29 +475,31 @@ __global__ void __launch_bounds__(Cfg<CG, BN>::THREADS, 1) gemm_e4m3_kernel(cons
     }
 }
 
-template <int CG, int BN>
+template <int CG, int BN, bool W8>
 cudaError_t launch_cfg(const GemmArgs& args, int units, cudaStream_t stream) {
-    using C = Cfg<CG, BN>;
+    using C = Cfg<CG, BN, W8>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_done[dev]) {
-        e = cudaFuncSetAttribute(gemm_e4m3_kernel<CG, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(gemm_e4m3_kernel<CG, BN, W8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    return launch_pdl(gemm_e4m3_kernel<CG, BN>, dim3((unsigned)(units * CG)), dim3(C::THREADS), C::SMEM_BYTES,
+    return launch_pdl(gemm_e4m3_kernel<CG, BN, W8>, dim3((unsigned)(units * CG)), dim3(C::THREADS), C::SMEM_BYTES,
                       stream, CG, args);
 }
 
 }  // namespace
 
-int gemm_block_m(int cfg) { return cfg == kCfgPair256 ? 256 : 128; }
-int gemm_block_n(int cfg) { return cfg == kCfg128x128 ? 128 : 256; }
+int gemm_block_m(int cfg) { return (cfg == kCfgPair256 || cfg == kCfgW8Pair256) ? 256 : 128; }
+int gemm_block_n(int cfg) { return (cfg == kCfg128x128 || cfg == kCfgW8128x128) ? 128 : 256; }
 int gemm_b_box_rows(int cfg) { return cfg == kCfg128x256 ? 256 : 128; }
-int gemm_cta_group(int cfg) { return cfg == kCfgPair256 ? 2 : 1; }
+int gemm_cta_group(int cfg) { return (cfg == kCfgPair256 || cfg == kCfgW8Pair256) ? 2 : 1; }
+bool gemm_weight_only(int cfg) { return cfg == kCfgW8Pair256 || cfg == kCfgW8128x128; }
+int gemm_k_elems(int cfg) { return gemm_weight_only(cfg) ? 64 : 128; }
 
 // MMA units (CTA pairs or CTAs) to launch: one per tile, at most one per SM (pair).
 int gemm_units_for(int cfg, int num_tiles, const DeviceInfo* dev) {
@@ -432,11 +510,15 @@ int gemm_units_for(int cfg, int num_tiles, const DeviceInfo* dev) {
 cudaError_t launch_gemm(int cfg, const GemmArgs& args, int units, cudaStream_t stream) {
     switch (cfg) {
         case kCfgPair256:
-            return launch_cfg<2, 256>(args, units, stream);
+            return launch_cfg<2, 256, false>(args, units, stream);
         case kCfg128x256:
-            return launch_cfg<1, 256>(args, units, stream);
+            return launch_cfg<1, 256, false>(args, units, stream);
         case kCfg128x128:
-            return launch_cfg<1, 128>(args, units, stream);
+            return launch_cfg<1, 128, false>(args, units, stream);
+        case kCfgW8Pair256:
+            return launch_cfg<2, 256, true>(args, units, stream);
+        case kCfgW8128x128:
+            return launch_cfg<1, 128, true>(args, units, stream);
         default:
             return cudaErrorInvalidValue;
     }

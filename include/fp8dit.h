@@ -180,6 +180,18 @@ fp8dit_status fp8_scaled_linear(fp8dit_linear h, int64_t M, const uint16_t* a_bf
                                 float* sa_scratch, uint16_t* y, fp8dit_stream_t stream);
 
 /*
+ * FP8 weight-only linear: the "FP8 weight-only scaled" pipeline the
+ * longcat-avatar-compare page sets against NVFP4 W4A4 (section 速度总览). The
+ * activation is not quantised; the layer's E4M3 weight is decoded to bf16 in
+ * shared memory and multiplied on the BF16 tensor cores:
+ *   y[m, n] = bf16_rne( (sum_k A[m,k] dec(qw[n,k])) * sw[n] + bias[n] ), fp32 accumulation.
+ *   a_bf16 [M, K] bf16 contiguous, y [M, N] bf16 contiguous, both 16-byte aligned.
+ * Uses the same handle (qw, sw, bias) as fp8_scaled_linear.
+ */
+fp8dit_status fp8_weight_only_linear(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, uint16_t* y,
+                                     fp8dit_stream_t stream);
+
+/*
  * fp8_scaled_linear from a bf16 activation, for callers that cannot allocate
  * device memory. The pages have no counterpart: this entry exists for code
  * that has no way to hand the library qa / sa scratch, such as a plugin whose

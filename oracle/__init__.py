@@ -10,6 +10,8 @@ What it computes (see oracle.c for the page citations):
   * ``quantize_tensor``: the same with one amax per tensor.
   * ``linear``: exact integer dot of dequantised E4M3 operands, then
     y = dot * sa[m] * sw[n] + bias[n] in double.
+  * ``linear_weight_only``: bf16 activation x decoded E4M3 weight, per-channel
+    scale and bias, in double.
   * ``act_bf16``: the producer activation (GELU erf / tanh form, SiLU) in
     double, rounded once to bf16.
 """
@@ -63,6 +65,8 @@ def _load():
         lib.or_linear.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p]
         lib.or_linear_at.restype = None
         lib.or_linear_at.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _p, _i64, _p]
+        lib.or_linear_weight_only.restype = None
+        lib.or_linear_weight_only.argtypes = [_p, _p, _p, _p, _i64, _i64, _i64, _p]
         lib.or_act.restype = ctypes.c_double
         lib.or_act.argtypes = [ctypes.c_int, ctypes.c_double]
         lib.or_round_bf16.restype = ctypes.c_uint16
@@ -128,6 +132,19 @@ def linear(qa, sa, qw, sw, bias=None) -> np.ndarray:
     y = np.empty((M, N), dtype=np.float64)
     _load().or_linear(qa.ctypes.data, sa.ctypes.data, qw.ctypes.data, sw.ctypes.data,
                       None if b is None else b.ctypes.data, M, N, K, y.ctypes.data)
+    return y
+
+
+def linear_weight_only(a, qw, sw, bias=None) -> np.ndarray:
+    """bf16 activation x E4M3 weight (decoded), per-channel scale, bias, in double."""
+    a, qw, sw = _c(a, np.uint16), _c(qw, np.uint8), _c(sw, np.float32)
+    M, K = a.shape
+    N = qw.shape[0]
+    assert qw.shape[1] == K and sw.shape == (N,)
+    b = None if bias is None else _c(bias, np.uint16)
+    y = np.empty((M, N), dtype=np.float64)
+    _load().or_linear_weight_only(a.ctypes.data, qw.ctypes.data, sw.ctypes.data,
+                                  None if b is None else b.ctypes.data, M, N, K, y.ctypes.data)
     return y
 
 

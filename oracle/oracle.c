@@ -207,6 +207,34 @@ void or_dot_units(const uint8_t* qa, const uint8_t* qw, int64_t M, int64_t N, in
         }
 }
 
+/* ----------------------------------------------------- FP8 weight-only linear */
+/*
+ * The "FP8 weight-only scaled" pipeline compared on the longcat-avatar-compare
+ * page (section 速度总览): the activation stays bf16, only the weight is FP8
+ * with its per-channel scale.
+ *   y[m, n] = (sum_k A[m,k] dec(qw[n,k])) * sw[n] + bias[n], in double.
+ * Every product of a bf16 value (8 significant bits) and an E4M3 value (4) is
+ * exact in double; the sum is plain double accumulation in k order.
+ */
+void or_linear_weight_only(const uint16_t* a, const uint8_t* qw, const float* sw, const uint16_t* bias,
+                           int64_t M, int64_t N, int64_t K, double* y) {
+    double wv[256];
+    for (int c = 0; c < 256; ++c) {
+        double v = or_decode(OR_E4M3FN, (uint8_t)c);
+        wv[c] = isnan(v) ? 0.0 : v;
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double dot = 0.0;
+            for (int64_t k = 0; k < K; ++k) dot += (double)or_bf16_to_f32(a[m * K + k]) * wv[qw[n * K + k]];
+            double v = dot * (double)sw[n];
+            if (bias) v += (double)or_bf16_to_f32(bias[n]);
+            y[m * N + n] = v;
+        }
+    }
+}
+
 /* ----------------------------------------------------- producer activations */
 /*
  * "从 BF16 到 FP8：HunyuanVideo1.5推理优化复盘", section 三.5: the GELU / SiLU that

@@ -100,3 +100,21 @@ def test_tolerance_helper():
     assert ok
     bad, _ = oracle.tolerance_ok(ref * (1 + 0.02), ref)
     assert not bad
+
+
+def test_weight_only_matches_float64_matmul_and_closed_form():
+    """The weight-only oracle against numpy's float64 matmul of the values
+    decoded by PyTorch (products exact; sums agree to double rounding), and a
+    closed form with constant operands."""
+    a = synth.normal_bf16("test/wo/a", (7, 96), 1.5)
+    qw = random_codes((5, 96), 11)
+    sw = np.linspace(0.5, 2.0, 5).astype(np.float32)
+    bias = synth.normal_bf16("test/wo/b", (5,), 0.1)
+    y = oracle.linear_weight_only(a, qw, sw, bias)
+    av = synth.bf16_to_f32(a).astype(np.float64)
+    ref = (av @ torch_decode(qw).T) * sw.astype(np.float64)[None, :] + synth.bf16_to_f32(bias).astype(np.float64)[None, :]
+    assert np.allclose(y, ref, rtol=1e-14, atol=1e-12)
+    ones = np.full((2, 64), 0x3F80, dtype=np.uint16)  # 1.0
+    qc = np.full((3, 64), 0x40, dtype=np.uint8)       # 2.0
+    y1 = oracle.linear_weight_only(ones, qc, np.array([1.0, 0.5, 0.25], dtype=np.float32))
+    assert np.array_equal(y1, np.array([[128.0, 64.0, 32.0]] * 2))
