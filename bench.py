@@ -566,6 +566,23 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
         bms = time_region(torch, lambda i: torch.matmul(a16, w16.t()), 50, dev)
         btf = 2.0 * M * N * K / (bms * 1e-3) / 1e12
         out[f"bf16_torch_matmul_ffn_{name}"] = {"us": bms * 1e3, "tflops": btf}
+    # Stream-K against the tile-per-pair schedule where the latter's last wave
+    # is nearly empty: 4864 tokens x FFN-down weight = 152 tiles on 74 pairs.
+    d = synth.ffn_down()
+    M, N, K = 4864, 2048, 8192
+    layer = fp8.FP8Linear.from_weight(up(d["W"]), up(d["bias"]))
+    qs = [fp8.quantize_rowwise(up(synth.normal_bf16(f"bench/sk/A{i}", (M, K), 1.0, outlier_p=0.001,
+                                                        outlier_factor=20.0))) for i in range(3)]
+    ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    run = lambda i: layer.forward_fp8(qs[i % 3][0], qs[i % 3][1], y=ys[i % 3])
+    dp_ms = time_region(torch, run, 100, dev)
+    layer.attach_workspace()
+    sk_ms = time_region(torch, run, 100, dev)
+    layer.detach_workspace()
+    out["stream_k_4864x2048x8192"] = {"tiles": 152, "pairs": 74, "plain_us": dp_ms * 1e3, "stream_k_us": sk_ms * 1e3,
+                                      "stream_k_tflops": 2.0 * M * N * K / (sk_ms * 1e-3) / 1e12,
+                                      "speedup": dp_ms / sk_ms}
+    del qs, ys, layer
     # State-dict conversion: 192 tensors, 1.61e9 elements, both formats.
     layout = synth.state_dict_layout()
     tensors = []

@@ -72,6 +72,9 @@ def load_library():
                                                  ctypes.c_size_t, p]
     L.fp8_linear_create.argtypes = [i64, i64, p, p, p, ctypes.c_int, ctypes.POINTER(p)]
     L.fp8_linear_destroy.argtypes = [p]
+    L.fp8_linear_workspace_size.argtypes = [p]
+    L.fp8_linear_workspace_size.restype = ctypes.c_size_t
+    L.fp8_linear_set_workspace.argtypes = [p, p, ctypes.c_size_t]
     L.fp8_scaled_linear.argtypes = [p, i64, p, p, p, p, p, p, p]
     L.fp8_scaled_linear_multi.argtypes = [ctypes.POINTER(p), i32, i64, p, p, p, ctypes.POINTER(p), p]
     L.fp8_scaled_linear_noalloc.argtypes = [p, i64, p, p, p]
@@ -85,7 +88,8 @@ def load_library():
                  "fp8_quantize_weight_per_tensor",
                  "fp8_linear_create", "fp8_linear_destroy", "fp8_scaled_linear", "fp8_scaled_linear_multi",
                  "fp8_scaled_linear_noalloc", "fp8_weight_only_linear",
-                 "fp8_linear_plan", "fp8dit_device_error", "fp8dit_selftest_expired_wait",
+                 "fp8_linear_plan", "fp8_linear_set_workspace", "fp8dit_device_error",
+                 "fp8dit_selftest_expired_wait",
                  "fp8dit_selftest_quotient"):
         getattr(L, name).restype = st
     _lib = L
@@ -279,6 +283,25 @@ class FP8Linear:
             self.close()
         except Exception:
             pass
+
+    def attach_workspace(self, workspace: Optional[torch.Tensor] = None) -> Optional[torch.Tensor]:
+        """Attach a stream-K workspace (allocated here when not given) and
+        return it, so that it can be attached to further layers whose calls
+        run one after another; detach_workspace() goes back to the plain
+        schedule."""
+        L = load_library()
+        need = int(L.fp8_linear_workspace_size(self._h))
+        if workspace is None:
+            workspace = torch.empty((need,), dtype=torch.uint8, device=self.device)
+        if workspace.numel() * workspace.element_size() < need or not workspace.is_cuda:
+            raise ValueError(f"workspace must be a CUDA tensor of at least {need} bytes")
+        _check(L.fp8_linear_set_workspace(self._h, workspace.data_ptr(), workspace.numel() * workspace.element_size()))
+        self.workspace = workspace  # keep it alive while attached
+        return workspace
+
+    def detach_workspace(self) -> None:
+        _check(load_library().fp8_linear_set_workspace(self._h, None, 0))
+        self.workspace = None
 
     def plan(self, M: int, n_problems: int = 1) -> Tuple[int, int, int]:
         bm, bn, ctas = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()

@@ -92,7 +92,24 @@ struct alignas(64) GemmArgs {
     int32_t num_tiles;
     int32_t num_kb;
     DevErr err;
+    // Stream-K schedule (pair FP8 configuration only): each MMA unit takes an
+    // equal contiguous share of the num_tiles x num_kb k-blocks. A tile split
+    // between units u and u+1 is finished by u: u+1 computes its k-block tail
+    // first, stores the fp32 partial in sk_partial and publishes sk_flag.
+    int32_t stream_k;
+    uint32_t sk_epoch;   // flag value that marks this launch's partials
+    uint32_t* sk_flag;   // [units][2 CTAs][8 epilogue warps]
+    float* sk_partial;   // [units][2 CTAs][8 epilogue warps][32 rows][128 columns]
 };
+
+// Bytes of stream-K workspace for `units` MMA units (flags, then partials).
+constexpr size_t kSkFlagBytesPerUnit = 2 * 8 * sizeof(uint32_t);
+constexpr size_t kSkPartialBytesPerUnit = 2 * 8 * 32 * 128 * sizeof(float);
+constexpr int64_t kSkMinKBlocks = 8;  // shorter tiles gain less from a split than it costs
+inline size_t stream_k_workspace_bytes(int units) {
+    const size_t flags = ((size_t)units * kSkFlagBytesPerUnit + 4095) & ~(size_t)4095;
+    return flags + (size_t)units * kSkPartialBytesPerUnit;
+}
 
 // Tile configurations the plan chooses from.
 enum GemmConfig : int32_t {

@@ -86,6 +86,63 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
     return TileCoord{g, local % a.tiles_m, local / a.tiles_m};
 }
 
+// The work of one MMA unit as a sequence of segments (tile t, k-blocks
+// [k0, k1)). Data-parallel: whole tiles unit, unit + units, ... Stream-K: the
+// unit's equal share [pos, end) of the num_tiles x num_kb k-blocks, cut at
+// tile boundaries. With num_tiles >= units a share spans at least one tile,
+// so a tile has at most two segments: a head [0, a) that ends its unit's
+// share and a tail [a, num_kb) that starts the next unit's share.
+struct Segment {
+    int t, k0, k1;
+};
+struct SegSched {
+    int64_t pos, end;
+    int step, num_kb;
+    bool sk;
+};
+__device__ __forceinline__ SegSched seg_begin(const GemmArgs& a, int unit, int units) {
+    SegSched s;
+    s.sk = a.stream_k != 0;
+    s.num_kb = a.num_kb;
+    if (s.sk) {
+        const int64_t total = (int64_t)a.num_tiles * a.num_kb;
+        s.pos = total * unit / units;
+        s.end = total * (unit + 1) / units;
+        s.step = 0;
+    } else {
+        s.pos = unit;
+        s.end = a.num_tiles;
+        s.step = units;
+    }
+    return s;
+}
+__device__ __forceinline__ bool seg_next(SegSched& s, Segment& g) {
+    if (s.pos >= s.end) return false;
+    if (s.sk) {
+        g.t = (int)(s.pos / s.num_kb);
+        g.k0 = (int)(s.pos % s.num_kb);
+        const int64_t tile_end = (int64_t)(g.t + 1) * s.num_kb;
+        const int64_t stop = tile_end < s.end ? tile_end : s.end;
+        g.k1 = g.k0 + (int)(stop - s.pos);
+        s.pos = stop;
+    } else {
+        g.t = (int)s.pos;
+        g.k0 = 0;
+        g.k1 = s.num_kb;
+        s.pos += s.step;
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu_u32(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -167,11 +224,13 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
             int64_t armed = 0;
-            for (int t = unit; t < args.num_tiles && !aborted; t += units) {
-                const TileCoord tc = tile_coord(args, t);
+            SegSched ss = seg_begin(args, unit, units);
+            Segment sg;
+            while (!aborted && seg_next(ss, sg)) {
+                const TileCoord tc = tile_coord(args, sg.t);
                 const int a_row = tc.tm * C::BM + (int)rank * C::ROWS;
                 const int b_row = tc.tn * BN + (int)rank * C::B_ROWS;
-                for (int kb = 0; kb < args.num_kb; ++kb) {
+                for (int kb = sg.k0; kb < sg.k1; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.err)) {
                         aborted = true;
                         abort_peer();
@@ -215,7 +274,9 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
         if (lane == 0 && leader) {
             constexpr uint32_t idesc = W8 ? umma_idesc_bf16_f32(C::BM, BN) : umma_idesc_e4m3_f32(C::BM, BN);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-            for (int t = unit; t < args.num_tiles && !aborted; t += units) {
+            SegSched ss = seg_begin(args, unit, units);
+            Segment sg;
+            while (!aborted && seg_next(ss, sg)) {
                 if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, args.err)) {
                     aborted = true;
                     abort_peer();
@@ -223,7 +284,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
-                for (int kb = 0; kb < args.num_kb; ++kb) {
+                for (int kb = sg.k0; kb < sg.k1; ++kb) {
                     // W8: the decoded B of both CTAs (and, through the decoders'
                     // waits, both CTAs' A) is ready. FP8: both CTAs' TMA loads landed.
                     if (!mbar_wait_bounded(W8 ? &conv[stage] : &full[stage], phase, abort_flag, args.err)) {
@@ -238,12 +299,13 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                     for (int j = 0; j < C::ROW_BYTES / 32; ++j) {  // 32 bytes of K per MMA
                         const uint64_t ad = umma_desc_kmajor_sw128(a0 + 32 * j);
                         const uint64_t bd = umma_desc_kmajor_sw128(b0 + 32 * j);
+                        const uint32_t accum = (kb > sg.k0 || j > 0) ? 1u : 0u;  // a segment starts a new sum
                         if (W8) {
-                            if (CG == 2) mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | j) != 0);
-                            else mma_bf16(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                            if (CG == 2) mma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+                            else mma_bf16(d_tmem, ad, bd, idesc, accum);
                         } else {
-                            if (CG == 2) mma_f8f6f4_pair(d_tmem, ad, bd, idesc, (kb | j) != 0);
-                            else mma_f8f6f4(d_tmem, ad, bd, idesc, (kb | j) != 0);
+                            if (CG == 2) mma_f8f6f4_pair(d_tmem, ad, bd, idesc, accum);
+                            else mma_f8f6f4(d_tmem, ad, bd, idesc, accum);
                         }
                     }
                     // The ring slot is free (in both CTAs) once these MMAs have read it.
@@ -331,15 +393,63 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
         uint32_t acc = 0, acc_phase = 0;
         uint32_t stores = 0;
         Pre pre;
-        if (unit < args.num_tiles) fetch(unit, pre);
-        for (int t = unit; t < args.num_tiles; t += units) {
-            const TileCoord tc = tile_coord(args, t);
+        SegSched ss = seg_begin(args, unit, units);
+        SegSched look = ss;  // one segment ahead, for the operand prefetch
+        Segment sg, nx;
+        bool has_next = seg_next(look, nx);
+        if (has_next) fetch(nx.t, pre);
+        while (seg_next(ss, sg)) {
+            has_next = seg_next(look, nx);
+            const TileCoord tc = tile_coord(args, sg.t);
             __syncwarp();  // every lane is done reading the previous tile's copy
             publish(pre);
             const float sa = pre.sa;
             __syncwarp();
-            if (t + units < args.num_tiles) fetch(t + units, pre);
+            if (has_next) fetch(nx.t, pre);
             const int row0 = tc.tm * C::BM + (int)rank * C::ROWS + q * 32;  // first row of this warp's box
+            // Stream-K roles of this segment: a tail stores its fp32 partial for
+            // the unit that finishes the tile; a head adds that partial. A warp's
+            // partial (32 rows x EPI_COLS fp32) is stored lane-fastest: float4 v
+            // of row `lane` in column chunk c sits at [(c * 8 + v) * 32 + lane],
+            // so every warp access moves 512 contiguous bytes.
+            const bool tail = sg.k0 > 0;
+            const bool head = sg.k0 == 0 && sg.k1 < args.num_kb;
+            const size_t part_elems = 32 * C::EPI_COLS;
+            float4* my_part = nullptr;
+            const float4* their_part = nullptr;
+            if (tail || head) {
+                const int slot = tail ? unit : unit + 1;  // tail: this unit's first segment
+                const size_t idx = ((size_t)slot * 2 + rank) * C::EPI_WARPS + ew;
+                float* base = args.sk_partial + idx * part_elems;
+                if (tail) my_part = reinterpret_cast<float4*>(base) + lane;
+                else their_part = reinterpret_cast<const float4*>(base) + lane;
+            }
+            float4 pp[8];  // the head's partial for the next column chunk
+            if (head) {
+                // The partner unit wrote this partial in its first segment, long
+                // before this unit's last one; wait, bounded, for its flag, then
+                // fetch the first chunk while the accumulator is still being built.
+                const uint32_t* flag = args.sk_flag + ((size_t)(unit + 1) * 2 + rank) * C::EPI_WARPS + ew;
+                bool ok = ld_acquire_gpu_u32(flag) == args.sk_epoch;
+                if (!ok) {
+                    const unsigned long long t0 = globaltimer_ns();
+                    while (!(ok = ld_acquire_gpu_u32(flag) == args.sk_epoch)) {
+                        if (*abort_flag) break;
+                        if (globaltimer_ns() - t0 > args.err.limit_ns) {
+                            *abort_flag = 1;
+                            atomicOr(args.err.word, kDevErrTimeout);
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                }
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) abort_peer();
+                    break;
+                }
+#pragma unroll
+                for (int v = 0; v < 8; ++v) pp[v] = __ldcg(their_part + v * 32);
+            }
 
             // Every lane waits; the warp then agrees (and reconverges) before
             // the warp-collective TMEM loads.
@@ -358,6 +468,29 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_addr + c * 32, r);
                 tmem_wait_ld();
+                if (tail) {
+                    // Raw fp32 accumulator of this piece: row `lane`, columns c*32..+31.
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        __stcg(my_part + (c * 8 + v) * 32,
+                               make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+                    continue;
+                }
+                if (head) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + pp[v].x);
+                        r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + pp[v].y);
+                        r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + pp[v].z);
+                        r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + pp[v].w);
+                    }
+                    // Next chunk's partial, in flight while this one is packed and stored.
+                    if (c + 1 < C::EPI_COLS / 32) {
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) pp[v] = __ldcg(their_part + ((c + 1) * 8 + v) * 32);
+                    }
+                }
                 uint32_t packed[16];
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
@@ -390,6 +523,13 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                 }
                 ++stores;
             }
+            if (tail) {
+                // Publish the partial: every lane's stores, then the flag.
+                __threadfence();
+                __syncwarp();
+                if (lane == 0)
+                    st_release_gpu_u32(args.sk_flag + ((size_t)unit * 2 + rank) * C::EPI_WARPS + ew, args.sk_epoch);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -414,8 +554,10 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
             const int ct = threadIdx.x - 32 * (2 + C::EPI_WARPS);
             uint32_t stage = 0, phase = 0;
             bool stop = false;
-            for (int t = unit; t < args.num_tiles && !stop; t += units) {
-                for (int kb = 0; kb < args.num_kb; ++kb) {
+            SegSched ss = seg_begin(args, unit, units);
+            Segment sg;
+            while (!stop && seg_next(ss, sg)) {
+                for (int kb = sg.k0; kb < sg.k1; ++kb) {
                     const bool ok = mbar_wait_bounded(&full[stage], phase, abort_flag, args.err);
                     if (!__all_sync(0xffffffffu, ok)) {
                         if (lane == 0) abort_peer();

@@ -164,6 +164,27 @@ fp8dit_status fp8_linear_create(int64_t N, int64_t K, const uint8_t* qw, const f
 fp8dit_status fp8_linear_destroy(fp8dit_linear h);
 
 /*
+ * Optional stream-K workspace for a layer. When a layer's 256 x 256 output
+ * tiles would keep the CTA pairs busy for less than 3/4 of the waves of a
+ * tile-per-pair schedule (a nearly empty last wave: e.g. 150 tiles on 74
+ * pairs) and a tile has at least 8 k-blocks of 128, each pair instead takes
+ * an equal share of the layer's k-blocks; a tile split between two pairs is
+ * finished by one of them after the other has stored its fp32 partial in this
+ * workspace. Results stay deterministic (the two parts are added once, in
+ * fp32) but differ in rounding from the plain schedule. Without a workspace,
+ * or for other shapes (the FFN shapes among them), the plain schedule is used.
+ *   fp8_linear_workspace_size: bytes needed on the layer's device (~19 MB on
+ *     148 SMs), the same for every M.
+ *   fp8_linear_set_workspace: attach caller-owned DEVICE memory (256-byte
+ *     aligned, at least that size) or detach with NULL. Attaching clears the
+ *     workspace's flags (synchronously). The workspace may be attached to
+ *     several layers whose calls run one after another on the GPU; calls that
+ *     overlap on the GPU must not share a workspace.
+ */
+size_t fp8_linear_workspace_size(fp8dit_linear h);
+fp8dit_status fp8_linear_set_workspace(fp8dit_linear h, void* workspace, size_t bytes);
+
+/*
  * Forward of one FP8 linear layer ("从 BF16 到 FP8", sections 三.1, 三.3, 三.5):
  *  - ordinary tensor: a_bf16 != NULL. A [M, K] bf16 (contiguous) is quantised
  *    per token into qa_scratch [M, K] and sa_scratch [M] (both caller-owned,
