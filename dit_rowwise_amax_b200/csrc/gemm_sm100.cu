@@ -51,14 +51,16 @@ struct Cfg {
     static constexpr int B_ROWS = BN / CG;  // W rows per CTA per stage
     static constexpr int A_BYTES = ROWS * ROW_BYTES;
     static constexpr int B_BYTES = B_ROWS * ROW_BYTES;         // MMA-ready B: FP8, or bf16 decoded from FP8
-    static constexpr int RAW_BYTES = W8 ? B_ROWS * 64 : 0;      // FP8 weight codes as loaded (W8 only)
+    // W8: the FP8 weight codes as loaded (B_ROWS rows x 64 bytes) land in the
+    // upper half of the stage's B buffer and are decoded in place.
+    static constexpr int RAW_BYTES = W8 ? B_ROWS * 64 : 0;
     static constexpr int TX_BYTES = A_BYTES + (W8 ? RAW_BYTES : B_BYTES);  // TMA bytes per CTA per stage
-    static constexpr int STAGE_SMEM = A_BYTES + B_BYTES + RAW_BYTES;
-    static constexpr int STAGES = W8 ? (B_ROWS == 256 ? 3 : 5) : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6));
+    static constexpr int STAGE_SMEM = A_BYTES + B_BYTES;
+    static constexpr int STAGES = W8 ? 6 : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6));
     static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
     static constexpr int EPI_WARPS = W8 ? 4 : 8;     // one or two per TMEM lane quarter
-    static constexpr int CONV_WARPS = W8 ? 4 : 0;    // FP8 -> bf16 weight decoders (W8)
+    static constexpr int CONV_WARPS = W8 ? STAGES : 0;  // FP8 -> bf16 weight decoders, one per stage (W8)
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
     static constexpr int BOX = 32;                   // epilogue store box: 32 rows x 32 columns
     static constexpr int STG_BYTES = BOX * BOX * 2;  // 2 KB, 64-byte rows, one per epilogue warp
@@ -71,6 +73,7 @@ struct Cfg {
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
     static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(!W8 || (B_BYTES == 2 * RAW_BYTES && B_ROWS == 128), "in-place decode layout");
 };
 
 struct TileCoord {
@@ -156,8 +159,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = sA + C::STAGES * C::A_BYTES;
-    uint8_t* sRaw = sB + C::STAGES * C::B_BYTES;
-    uint8_t* staging = sRaw + C::STAGES * C::RAW_BYTES;
+    uint8_t* staging = sB + C::STAGES * C::B_BYTES;
     float* swb = reinterpret_cast<float*>(staging + C::STAGING_BYTES);
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(swb) + C::SWB_BYTES);
     uint64_t* empty = full + C::STAGES;
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&conv[s], C::CONV_WARPS * CG > 0 ? C::CONV_WARPS * CG : 1);
+            mbar_init(&conv[s], CG);  // the stage's decoder warp in each CTA (W8)
         }
         for (int a = 0; a < C::ACC; ++a) {
             mbar_init(&tfull[a], 1);
@@ -241,7 +243,8 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                         // decoder warps wait on them.
                         mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
                         tma_load_2d(sA + stage * C::A_BYTES, &args.tmA, &full[stage], kb * C::KE, a_row);
-                        tma_load_2d(sRaw + stage * C::RAW_BYTES, &args.tmB[tc.g], &full[stage], kb * C::KE, b_row);
+                        tma_load_2d(sB + stage * C::B_BYTES + C::RAW_BYTES, &args.tmB[tc.g], &full[stage],
+                                    kb * C::KE, b_row);
                     } else if (CG == 2) {
                         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
                         if (leader) mbar_arrive_expect_tx(&full[stage], CG * C::TX_BYTES);
@@ -545,50 +548,71 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ FP8 -> bf16 weight decoders (W8)
-        // Stage s: sRaw holds B_ROWS rows x 64 FP8 codes (64-byte rows, as
-        // loaded); write them as B_ROWS rows x 64 bf16 (128-byte rows, 128-byte
-        // swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)), the
-        // K-major layout the MMA descriptors describe. E4M3 values are exact
-        // in bf16. Then release the stage to the pair leader's MMA.
+        // Decoder warp s owns ring stage s, so it waits on that stage's
+        // barrier phase after phase, and STAGES stages are decoded, fenced and
+        // released concurrently. The stage's B buffer (B_ROWS rows of 128
+        // bytes) holds, in its upper half, the FP8 codes as loaded (B_ROWS
+        // rows of 64 bytes). They are decoded in place into B_ROWS rows x 64
+        // bf16 with the 128-byte swizzle (16-byte chunk c of row r at chunk
+        // c ^ (r & 7)), the K-major layout the MMA descriptors describe; E4M3
+        // values are exact in bf16. Rows go in batches of kRowsPerBatch, each
+        // read whole before any of it is written: writing decoded rows
+        // [r0, r1) covers code rows below 2 * r1 - B_ROWS <= r1, all read
+        // already, so no code is overwritten before it is decoded.
         if constexpr (W8) {
-            const int ct = threadIdx.x - 32 * (2 + C::EPI_WARPS);
+            constexpr int kIters = 4;                      // 16-byte code chunks per lane per batch
+            constexpr int kRowsPerBatch = kIters * 32 / 4;  // 4 chunks per 64-byte code row
+            const int own = warp - (2 + C::EPI_WARPS);     // the stage this warp decodes
             uint32_t stage = 0, phase = 0;
             bool stop = false;
             SegSched ss = seg_begin(args, unit, units);
             Segment sg;
             while (!stop && seg_next(ss, sg)) {
                 for (int kb = sg.k0; kb < sg.k1; ++kb) {
-                    const bool ok = mbar_wait_bounded(&full[stage], phase, abort_flag, args.err);
-                    if (!__all_sync(0xffffffffu, ok)) {
-                        if (lane == 0) abort_peer();
-                        stop = true;
-                        break;
-                    }
-                    const uint8_t* raw = sRaw + stage * C::RAW_BYTES;
-                    uint8_t* dst = sB + stage * C::B_BYTES;
-#pragma unroll 2
-                    for (int idx = ct; idx < C::B_ROWS * 4; idx += 32 * C::CONV_WARPS) {
-                        const int r = idx >> 2, c = idx & 3;
-                        const uint4 v = *reinterpret_cast<const uint4*>(raw + r * 64 + c * 16);
-                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                        uint32_t o[8];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] & 0xffffu), __NV_E4M3);
-                            const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> 16), __NV_E4M3);
-                            o[2 * k] = pack_bf16x2(__half2float(__ushort_as_half(lo.x)), __half2float(__ushort_as_half(lo.y)));
-                            o[2 * k + 1] = pack_bf16x2(__half2float(__ushort_as_half(hi.x)), __half2float(__ushort_as_half(hi.y)));
+                    if ((int)stage == own) {
+                        const bool ok = mbar_wait_bounded(&full[stage], phase, abort_flag, args.err);
+                        if (!__all_sync(0xffffffffu, ok)) {
+                            if (lane == 0) abort_peer();
+                            stop = true;
+                            break;
                         }
-                        *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c) ^ (r & 7)) << 4)) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
-                        *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4)) =
-                            make_uint4(o[4], o[5], o[6], o[7]);
-                    }
-                    fence_proxy_async_smem();  // the tensor core reads these bytes through the async proxy
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&conv[stage]), 0));
-                        else mbar_arrive(&conv[stage]);
+                        uint8_t* dst = sB + stage * C::B_BYTES;
+                        const uint8_t* raw = dst + C::RAW_BYTES;
+#pragma unroll 1
+                        for (int r0 = 0; r0 < C::B_ROWS; r0 += kRowsPerBatch) {
+                            uint4 v[kIters];
+#pragma unroll
+                            for (int i = 0; i < kIters; ++i)
+                                v[i] = *reinterpret_cast<const uint4*>(raw + r0 * 64 + (i * 32 + lane) * 16);
+                            __syncwarp();  // the whole batch is read before any lane writes
+#pragma unroll
+                            for (int i = 0; i < kIters; ++i) {
+                                const int r = r0 + ((i * 32 + lane) >> 2), c = lane & 3;
+                                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+                                uint32_t o[8];
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const __half2_raw lo =
+                                        __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] & 0xffffu), __NV_E4M3);
+                                    const __half2_raw hi =
+                                        __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[k] >> 16), __NV_E4M3);
+                                    o[2 * k] = pack_bf16x2(__half2float(__ushort_as_half(lo.x)),
+                                                           __half2float(__ushort_as_half(lo.y)));
+                                    o[2 * k + 1] = pack_bf16x2(__half2float(__ushort_as_half(hi.x)),
+                                                               __half2float(__ushort_as_half(hi.y)));
+                                }
+                                *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c) ^ (r & 7)) << 4)) =
+                                    make_uint4(o[0], o[1], o[2], o[3]);
+                                *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4)) =
+                                    make_uint4(o[4], o[5], o[6], o[7]);
+                            }
+                        }
+                        fence_proxy_async_smem();  // the tensor core reads these bytes through the async proxy
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&conv[stage]), 0));
+                            else mbar_arrive(&conv[stage]);
+                        }
                     }
                     if (++stage == C::STAGES) {
                         stage = 0;
