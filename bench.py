@@ -552,6 +552,17 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
         tf = 2.0 * M * N * K / (ms * 1e-3) / 1e12
         out[f"gemm_only_ffn_{name}"] = {"us": ms * 1e3, "tflops": tf, "frac_of_fp8_peak": tf / fp8_peak,
                                         "plan": list(layer.plan(M))}
+        # Quantise-in-GEMM variant against quantiser + GEMM, both from bf16 A.
+        qa_s = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        sa_s = torch.empty((M,), dtype=torch.float32, device=dev)
+        sc_s = torch.empty((2 * M,), dtype=torch.float32, device=dev)
+        a16s = [up(d["A"]) for _ in range(3)]
+        fz_ms = time_region(torch, lambda i: layer.forward_fused(a16s[i % 3], y=ys[i % 3], scale_scratch=sc_s), 50, dev)
+        uf_ms = time_region(torch, lambda i: layer.forward(a16s[i % 3], y=ys[i % 3], qa_scratch=qa_s, sa_scratch=sa_s),
+                            50, dev)
+        out[f"quantize_in_gemm_ffn_{name}"] = {"fused_us": fz_ms * 1e3, "quantizer_plus_gemm_us": uf_ms * 1e3,
+                                              "tflops": 2.0 * M * N * K / (fz_ms * 1e-3) / 1e12}
+        del a16s, qa_s, sa_s, sc_s
         # FP8 weight-only (bf16 activation, E4M3 weight decoded in shared
         # memory, BF16 tensor cores), same layer.
         a16s = [up(d["A"]) for _ in range(3)]

@@ -79,6 +79,7 @@ def load_library():
     L.fp8_scaled_linear_multi.argtypes = [ctypes.POINTER(p), i32, i64, p, p, p, ctypes.POINTER(p), p]
     L.fp8_scaled_linear_noalloc.argtypes = [p, i64, p, p, p]
     L.fp8_weight_only_linear.argtypes = [p, i64, p, p, p]
+    L.fp8_scaled_linear_fused.argtypes = [p, i64, p, p, p, p]
     L.fp8_linear_plan.argtypes = [p, i64, i32, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.fp8dit_device_error.argtypes = [p]
     L.fp8dit_selftest_expired_wait.argtypes = [i64, p]
@@ -87,7 +88,7 @@ def load_library():
     for name in ("fp8_quantize_rowwise", "fp8_act_quantize_rowwise", "fp8_quantize_weight_per_channel",
                  "fp8_quantize_weight_per_tensor",
                  "fp8_linear_create", "fp8_linear_destroy", "fp8_scaled_linear", "fp8_scaled_linear_multi",
-                 "fp8_scaled_linear_noalloc", "fp8_weight_only_linear",
+                 "fp8_scaled_linear_noalloc", "fp8_weight_only_linear", "fp8_scaled_linear_fused",
                  "fp8_linear_plan", "fp8_linear_set_workspace", "fp8dit_device_error",
                  "fp8dit_selftest_expired_wait",
                  "fp8dit_selftest_quotient"):
@@ -338,6 +339,26 @@ class FP8Linear:
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.bfloat16, device=a.device)
         _check(load_library().fp8_weight_only_linear(self._h, M, a.data_ptr(), y.data_ptr(), _stream(a.device)))
+        return y
+
+    def forward_fused(self, a: torch.Tensor, y: Optional[torch.Tensor] = None,
+                      scale_scratch: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """The FP8 linear from a bf16 activation with the per-token quantisation
+        done inside the GEMM (a row-scale pre-pass, then bf16 tiles quantised
+        to E4M3 in shared memory); same codes and result as forward().
+        scale_scratch: float32 [2 * M] (scales, then their reciprocals)."""
+        a = _bf16_matrix(a, "a")
+        if not a.is_contiguous() or a.shape[1] != self.K:
+            raise ValueError(f"a must be contiguous [M, {self.K}]")
+        M = a.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.bfloat16, device=a.device)
+        if scale_scratch is None:
+            scale_scratch = torch.empty((2 * M,), dtype=torch.float32, device=a.device)
+        if scale_scratch.dtype != torch.float32 or scale_scratch.numel() < 2 * M or not scale_scratch.is_cuda:
+            raise ValueError("scale_scratch must be a CUDA float32 tensor of at least 2 * M elements")
+        _check(load_library().fp8_scaled_linear_fused(self._h, M, a.data_ptr(), scale_scratch.data_ptr(),
+                                                      y.data_ptr(), _stream(a.device)))
         return y
 
     def forward_fp8(self, qa: torch.Tensor, sa: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -203,21 +203,36 @@ static int choose_cfg_weight_only(const fp8dit_linear_s* h, int64_t M) {
     return kCfgW8128x128;
 }
 
+// Quantise-in-GEMM plan: the same choice between pair tiles and 128 x 128 tiles.
+static int choose_cfg_fused(const fp8dit_linear_s* h, int64_t M) {
+    const int pairs = h->num_sms / 2;
+    if (M >= 256 && tiles_for(h, M, 1, kCfgAQPair256) * 2 >= pairs) return kCfgAQPair256;
+    return kCfgAQ128x128;
+}
+
 // a: FP8 codes [M, K] (qa) for the FP8 x FP8 configurations, bf16 [M, K] for
 // the weight-only ones; sa: per-token scales, or NULL (weight-only).
 static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, const void* a, const float* sa,
-                              uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev, int cfg) {
+                              uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev, int cfg,
+                              const float* ra = nullptr) {
     const int bm = gemm_block_m(cfg);
     const int bn = gemm_block_n(cfg);
     const int ke = gemm_k_elems(cfg);
     const int64_t K = hs[0]->K;
     GemmArgs args;
     memset(&args, 0, sizeof(args));
-    fp8dit_status st = gemm_weight_only(cfg)
-                           ? encode_tma_2d(&args.tmA, 2, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, (uint32_t)ke,
-                                           128, CU_TENSOR_MAP_SWIZZLE_128B)
-                           : encode_tma_2d(&args.tmA, 1, a, (uint64_t)K, (uint64_t)M, (uint64_t)K, (uint32_t)ke,
-                                           128, CU_TENSOR_MAP_SWIZZLE_128B);
+    // A: FP8 codes (128-byte rows, swizzled, MMA-ready); weight-only: bf16
+    // (128-byte rows of 64 elements, swizzled, MMA-ready); quantise-in-GEMM:
+    // bf16 rows of 128 elements (256 bytes, unswizzled), quantised in shared memory.
+    fp8dit_status st =
+        gemm_weight_only(cfg)
+            ? encode_tma_2d(&args.tmA, 2, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, (uint32_t)ke, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B)
+        : gemm_quantizes_a(cfg)
+            ? encode_tma_2d(&args.tmA, 2, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, (uint32_t)ke, 128,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)
+            : encode_tma_2d(&args.tmA, 1, a, (uint64_t)K, (uint64_t)M, (uint64_t)K, (uint32_t)ke, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FP8DIT_OK) return st;
     const int tiles_m = (int)((M + bm - 1) / bm);
     int tiles = 0;
@@ -255,6 +270,7 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
         }
     }
     args.sa = sa;
+    args.ra = ra;
     args.M = (int32_t)M;
     args.K = (int32_t)hs[0]->K;
     args.G = n;
@@ -499,6 +515,28 @@ fp8dit_status fp8_weight_only_linear(fp8dit_linear h, int64_t M, const uint16_t*
     const DeviceInfo* dev = device_info();
     if (!dev) return FP8DIT_ERR_CUDA;
     return run_gemm(&h, 1, M, a_bf16, nullptr, &y, (cudaStream_t)stream, dev, choose_cfg_weight_only(h, M));
+}
+
+fp8dit_status fp8_scaled_linear_fused(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, float* scale_scratch,
+                                      uint16_t* y, fp8dit_stream_t stream) {
+    t_last_error[0] = 0;
+    if (!h) return invalid("null handle");
+    if (M < 0) return invalid("M must be >= 0");
+    if (M > kMaxRows) return unsupported("M too large");
+    if (M == 0) return FP8DIT_OK;
+    if (!a_bf16 || !aligned16(a_bf16)) return invalid("a_bf16 must be non-null and 16-byte aligned");
+    if (!scale_scratch || ((uintptr_t)scale_scratch & 3u) != 0)
+        return invalid("scale_scratch must be non-null and 4-byte aligned");
+    if (!y || !aligned16(y)) return invalid("y must be non-null and 16-byte aligned");
+    fp8dit_status st = check_device(h);
+    if (st != FP8DIT_OK) return st;
+    const DeviceInfo* dev = device_info();
+    if (!dev) return FP8DIT_ERR_CUDA;
+    float* sa = scale_scratch;
+    float* ra = scale_scratch + M;
+    cudaError_t e = launch_row_scales(a_bf16, M, h->K, h->K, sa, ra, (cudaStream_t)stream, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "row scale launch");
+    return run_gemm(&h, 1, M, a_bf16, sa, &y, (cudaStream_t)stream, dev, choose_cfg_fused(h, M), ra);
 }
 
 fp8dit_status fp8_scaled_linear_multi(const fp8dit_linear* hs, int32_t n, int64_t M, const uint16_t* a_bf16,

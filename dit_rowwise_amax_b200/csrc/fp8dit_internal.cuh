@@ -53,6 +53,11 @@ fp8dit_status encode_tma_2d(CUtensorMap* map, int elem_bytes, const void* base, 
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int fmt,
                                  uint8_t* q, int64_t ldq, float* scale, cudaStream_t stream,
                                  const DeviceInfo* dev);
+// Per-row E4M3 scales S = amax / 448 (1 for an all-zero row) and, where the
+// corrected-reciprocal quotient applies, rcp = RN(1 / S) (else 0): what the
+// rowwise quantiser uses, without writing codes.
+cudaError_t launch_row_scales(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float* scale, float* rcp,
+                              cudaStream_t stream, const DeviceInfo* dev);
 cudaError_t launch_act_quantize_rows(const uint16_t* h, int64_t M, int64_t K, int64_t ldh, int act, uint8_t* q,
                                      int64_t ldq, float* scale, uint16_t* g, int64_t ldg, cudaStream_t stream,
                                      const DeviceInfo* dev);
@@ -87,6 +92,7 @@ struct alignas(64) GemmArgs {
     CUtensorMap tmY[kMaxGroups];   // y bf16 [M, N], box 32 x 32, 64-byte swizzle (TMA store)
     GemmProblem prob[kMaxGroups];
     const float* sa;
+    const float* ra;  // AQ: RN(1 / sa[m]) where the corrected-reciprocal quotient applies, else 0
     int32_t M, K, G;
     int32_t tiles_m;
     int32_t num_tiles;
@@ -118,13 +124,16 @@ enum GemmConfig : int32_t {
     kCfg128x128 = 2,    // FP8 x FP8: 128 x 128 tile on one CTA
     kCfgW8Pair256 = 3,  // bf16 x FP8 weight (weight-only): 256 x 256 tile on a 2-CTA pair
     kCfgW8128x128 = 4,  // bf16 x FP8 weight (weight-only): 128 x 128 tile on one CTA
-    kNumCfgs = 5,
+    kCfgAQPair256 = 5,  // bf16 A quantised in the GEMM x FP8 weight: 256 x 256 tile on a 2-CTA pair
+    kCfgAQ128x128 = 6,  // bf16 A quantised in the GEMM x FP8 weight: 128 x 128 tile on one CTA
+    kNumCfgs = 7,
 };
 int gemm_block_m(int cfg);
 int gemm_block_n(int cfg);
 int gemm_b_box_rows(int cfg);
 int gemm_cta_group(int cfg);
 bool gemm_weight_only(int cfg);
+bool gemm_quantizes_a(int cfg);  // bf16 A quantised in the kernel (per-row scales sa, reciprocals ra)
 int gemm_k_elems(int cfg);  // K elements per pipeline stage
 constexpr int kGemmBlockK = 128;  // bytes = FP8 elements per k-block (one 128 B swizzle row)
 constexpr int kGemmStoreBox = 32;

@@ -37,30 +37,44 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include "fp8_codec.cuh"
 #include "fp8dit_internal.cuh"
 
 namespace fp8dit {
 namespace {
 
-template <int CG, int BN, bool W8>
+// Operand modes of the kernel.
+//   kOpsFp8: A and W are FP8 codes, both loaded by TMA (the FP8 linear).
+//   kOpsW8:  A is bf16; W codes are decoded to bf16 in shared memory (weight-only).
+//   kOpsAQ:  A is bf16 and is quantised to FP8 in shared memory with per-row
+//            scales computed beforehand; W is FP8 (quantise-in-GEMM variant).
+enum : int { kOpsFp8 = 0, kOpsW8 = 1, kOpsAQ = 2 };
+
+template <int CG, int BN, int OPS>
 struct Cfg {
+    static constexpr bool W8 = OPS == kOpsW8;
+    static constexpr bool AQ = OPS == kOpsAQ;
+    static constexpr bool CONV = W8 || AQ;  // has converter warps
     static constexpr int BM = 128 * CG;     // rows of one MMA tile
     static constexpr int ROWS = 128;        // rows per CTA (TMEM lanes)
     static constexpr int ROW_BYTES = 128;   // one 128-byte swizzle row per operand row per stage
     static constexpr int KE = W8 ? 64 : 128;  // K elements per stage (bf16 : FP8)
     static constexpr int B_ROWS = BN / CG;  // W rows per CTA per stage
-    static constexpr int A_BYTES = ROWS * ROW_BYTES;
+    static constexpr int A_BYTES = ROWS * ROW_BYTES;  // MMA-ready A per stage
+    // AQ: the bf16 A tile as loaded (ROWS rows x 256 bytes) fills the stage's
+    // A buffer and is quantised in place into its first A_BYTES.
+    static constexpr int A_STAGE = AQ ? 2 * A_BYTES : A_BYTES;
     static constexpr int B_BYTES = B_ROWS * ROW_BYTES;         // MMA-ready B: FP8, or bf16 decoded from FP8
     // W8: the FP8 weight codes as loaded (B_ROWS rows x 64 bytes) land in the
     // upper half of the stage's B buffer and are decoded in place.
     static constexpr int RAW_BYTES = W8 ? B_ROWS * 64 : 0;
-    static constexpr int TX_BYTES = A_BYTES + (W8 ? RAW_BYTES : B_BYTES);  // TMA bytes per CTA per stage
-    static constexpr int STAGE_SMEM = A_BYTES + B_BYTES;
-    static constexpr int STAGES = W8 ? 6 : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6));
+    static constexpr int TX_BYTES = A_STAGE + (W8 ? RAW_BYTES : B_BYTES);  // TMA bytes per CTA per stage
+    static constexpr int STAGE_SMEM = A_STAGE + B_BYTES;
+    static constexpr int STAGES = W8 ? 6 : AQ ? 4 : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6));
     static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
-    static constexpr int EPI_WARPS = W8 ? 4 : 8;     // one or two per TMEM lane quarter
-    static constexpr int CONV_WARPS = W8 ? STAGES : 0;  // FP8 -> bf16 weight decoders, one per stage (W8)
+    static constexpr int EPI_WARPS = CONV ? 4 : 8;   // one or two per TMEM lane quarter
+    static constexpr int CONV_WARPS = CONV ? STAGES : 0;  // converter warps, one per ring stage
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
     static constexpr int BOX = 32;                   // epilogue store box: 32 rows x 32 columns
     static constexpr int STG_BYTES = BOX * BOX * 2;  // 2 KB, 64-byte rows, one per epilogue warp
@@ -74,6 +88,7 @@ struct Cfg {
     static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(!W8 || (B_BYTES == 2 * RAW_BYTES && B_ROWS == 128), "in-place decode layout");
+    static_assert(!AQ || ROWS == 128, "in-place quantise layout");
 };
 
 struct TileCoord {
@@ -151,19 +166,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int CG, int BN, bool W8>
-__global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
+template <int CG, int BN, int OPS>
+__global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     gemm_e4m3_kernel(const __grid_constant__ GemmArgs args) {
-    using C = Cfg<CG, BN, W8>;
+    using C = Cfg<CG, BN, OPS>;
+    constexpr bool W8 = C::W8;
+    constexpr bool AQ = C::AQ;
+    constexpr bool CONV = C::CONV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = sA + C::STAGES * C::A_BYTES;
+    uint8_t* sB = sA + C::STAGES * C::A_STAGE;
     uint8_t* staging = sB + C::STAGES * C::B_BYTES;
     float* swb = reinterpret_cast<float*>(staging + C::STAGING_BYTES);
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(swb) + C::SWB_BYTES);
     uint64_t* empty = full + C::STAGES;
-    uint64_t* conv = empty + C::STAGES;  // W8: decoded B stage ready (arrivals from both CTAs' decoders)
+    uint64_t* conv = empty + C::STAGES;  // W8 / AQ: converted stage ready (arrivals from both CTAs' converters)
     uint64_t* tfull = conv + C::STAGES;
     uint64_t* tempty = tfull + C::ACC;
     uint64_t* drain = tempty + C::ACC;
@@ -186,7 +204,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&conv[s], CG);  // the stage's decoder warp in each CTA (W8)
+            mbar_init(&conv[s], CG);  // the stage's converter warp in each CTA (W8 / AQ)
         }
         for (int a = 0; a < C::ACC; ++a) {
             mbar_init(&tfull[a], 1);
@@ -238,21 +256,22 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                         abort_peer();
                         break;
                     }
-                    if (W8) {
-                        // Each CTA tracks its own bf16 A and FP8 W loads; its
-                        // decoder warps wait on them.
+                    if (CONV) {
+                        // Each CTA tracks its own A and W loads; its converter
+                        // warps wait on them. W8: the codes go to the upper half
+                        // of the B buffer (decoded in place).
                         mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-                        tma_load_2d(sA + stage * C::A_BYTES, &args.tmA, &full[stage], kb * C::KE, a_row);
-                        tma_load_2d(sB + stage * C::B_BYTES + C::RAW_BYTES, &args.tmB[tc.g], &full[stage],
+                        tma_load_2d(sA + stage * C::A_STAGE, &args.tmA, &full[stage], kb * C::KE, a_row);
+                        tma_load_2d(sB + stage * C::B_BYTES + (W8 ? C::RAW_BYTES : 0), &args.tmB[tc.g], &full[stage],
                                     kb * C::KE, b_row);
                     } else if (CG == 2) {
                         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
                         if (leader) mbar_arrive_expect_tx(&full[stage], CG * C::TX_BYTES);
-                        tma_load_2d_pair(sA + stage * C::A_BYTES, &args.tmA, bar, kb * C::KE, a_row);
+                        tma_load_2d_pair(sA + stage * C::A_STAGE, &args.tmA, bar, kb * C::KE, a_row);
                         tma_load_2d_pair(sB + stage * C::B_BYTES, &args.tmB[tc.g], bar, kb * C::KE, b_row);
                     } else {
                         mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-                        tma_load_2d(sA + stage * C::A_BYTES, &args.tmA, &full[stage], kb * C::KE, a_row);
+                        tma_load_2d(sA + stage * C::A_STAGE, &args.tmA, &full[stage], kb * C::KE, a_row);
                         tma_load_2d(sB + stage * C::B_BYTES, &args.tmB[tc.g], &full[stage], kb * C::KE, b_row);
                     }
                     ++armed;
@@ -262,7 +281,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                     }
                 }
             }
-            if (aborted && (leader || W8)) {
+            if (aborted && (leader || CONV)) {
                 // Let every copy signalled on this CTA's barriers land before exit.
                 for (int s = 0; s < C::STAGES; ++s) {
                     if (armed <= s) break;
@@ -288,15 +307,16 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 for (int kb = sg.k0; kb < sg.k1; ++kb) {
-                    // W8: the decoded B of both CTAs (and, through the decoders'
-                    // waits, both CTAs' A) is ready. FP8: both CTAs' TMA loads landed.
-                    if (!mbar_wait_bounded(W8 ? &conv[stage] : &full[stage], phase, abort_flag, args.err)) {
+                    // W8 / AQ: both CTAs' converted operands (and, through the
+                    // converters' waits, both CTAs' loads) are ready. FP8: both
+                    // CTAs' TMA loads landed.
+                    if (!mbar_wait_bounded(CONV ? &conv[stage] : &full[stage], phase, abort_flag, args.err)) {
                         aborted = true;
                         abort_peer();
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+                    const uint32_t a0 = smem_u32(sA + stage * C::A_STAGE);
                     const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
                     for (int j = 0; j < C::ROW_BYTES / 32; ++j) {  // 32 bytes of K per MMA
@@ -621,6 +641,77 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
                 }
             }
         }
+        if constexpr (AQ) {
+            // ------------------------------------------------ bf16 -> FP8 A quantisers (AQ)
+            // Converter warp s owns ring stage s. The stage's A buffer holds
+            // the tile's ROWS x 128 bf16 as loaded (256-byte rows, unswizzled);
+            // each row is quantised with its token's scale sa[m] and
+            // reciprocal ra[m] (written by the scale pre-pass from the row
+            // amax, exactly as the rowwise quantiser derives them) by the same
+            // code path as the rowwise quantiser, so the codes are identical.
+            // They are written in place as ROWS rows x 128 codes with the
+            // 128-byte swizzle. Rows go in batches of 16, each read whole
+            // before any of it is written: FP8 rows [r0, r0 + 16) cover bf16
+            // rows [r0 / 2, r0 / 2 + 8), all read already (or, for r0 = 0, in
+            // this batch). Rows at or beyond M are zeros (TMA fill) and get
+            // scale 1.
+            constexpr int kIters = 8;                        // 16-byte bf16 chunks per lane per batch
+            constexpr int kRowsPerBatch = kIters * 32 / 16;  // 16 chunks per 256-byte bf16 row
+            const int own = warp - (2 + C::EPI_WARPS);
+            uint32_t stage = 0, phase = 0;
+            bool stop = false;
+            SegSched ss = seg_begin(args, unit, units);
+            Segment sg;
+            while (!stop && seg_next(ss, sg)) {
+                const TileCoord tc = tile_coord(args, sg.t);
+                const int row_base = tc.tm * C::BM + (int)rank * C::ROWS;
+                for (int kb = sg.k0; kb < sg.k1; ++kb) {
+                    if ((int)stage == own) {
+                        const bool ok = mbar_wait_bounded(&full[stage], phase, abort_flag, args.err);
+                        if (!__all_sync(0xffffffffu, ok)) {
+                            if (lane == 0) abort_peer();
+                            stop = true;
+                            break;
+                        }
+                        uint8_t* buf = sA + stage * C::A_STAGE;
+#pragma unroll 1
+                        for (int r0 = 0; r0 < C::ROWS; r0 += kRowsPerBatch) {
+                            uint4 v[kIters];
+                            float sv[kIters], rv[kIters];
+#pragma unroll
+                            for (int i = 0; i < kIters; ++i) {
+                                const int idx = i * 32 + lane;  // chunk (idx & 15) of row r0 + (idx >> 4)
+                                v[i] = *reinterpret_cast<const uint4*>(buf + (r0 + (idx >> 4)) * 256 + (idx & 15) * 16);
+                                const int grow = row_base + r0 + (idx >> 4);
+                                sv[i] = grow < args.M ? __ldg(args.sa + grow) : 1.0f;
+                                rv[i] = grow < args.M ? __ldg(args.ra + grow) : 1.0f;
+                            }
+                            __syncwarp();  // the whole batch is read before any lane writes
+#pragma unroll
+                            for (int i = 0; i < kIters; ++i) {
+                                const int idx = i * 32 + lane;
+                                const int r = r0 + (idx >> 4), c16 = idx & 15;
+                                const Quot2 q2{f2_pack(rv[i], rv[i]), f2_pack(-sv[i], -sv[i]), sv[i]};
+                                const uint2 codes = rv[i] != 0.0f ? quant8<FP8DIT_E4M3FN, true>(v[i], q2)
+                                                                  : quant8<FP8DIT_E4M3FN, false>(v[i], q2);
+                                *reinterpret_cast<uint2*>(buf + r * 128 + (((c16 >> 1) ^ (r & 7)) << 4) +
+                                                          (c16 & 1) * 8) = codes;
+                            }
+                        }
+                        fence_proxy_async_smem();  // the tensor core reads these bytes through the async proxy
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&conv[stage]), 0));
+                            else mbar_arrive(&conv[stage]);
+                        }
+                    }
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
         __syncwarp();
     }
 
@@ -641,30 +732,33 @@ __global__ void __launch_bounds__(Cfg<CG, BN, W8>::THREADS, 1)
     }
 }
 
-template <int CG, int BN, bool W8>
+template <int CG, int BN, int OPS>
 cudaError_t launch_cfg(const GemmArgs& args, int units, cudaStream_t stream) {
-    using C = Cfg<CG, BN, W8>;
+    using C = Cfg<CG, BN, OPS>;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_done[dev]) {
-        e = cudaFuncSetAttribute(gemm_e4m3_kernel<CG, BN, W8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(gemm_e4m3_kernel<CG, BN, OPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    return launch_pdl(gemm_e4m3_kernel<CG, BN, W8>, dim3((unsigned)(units * CG)), dim3(C::THREADS), C::SMEM_BYTES,
+    return launch_pdl(gemm_e4m3_kernel<CG, BN, OPS>, dim3((unsigned)(units * CG)), dim3(C::THREADS), C::SMEM_BYTES,
                       stream, CG, args);
 }
 
 }  // namespace
 
-int gemm_block_m(int cfg) { return (cfg == kCfgPair256 || cfg == kCfgW8Pair256) ? 256 : 128; }
-int gemm_block_n(int cfg) { return (cfg == kCfg128x128 || cfg == kCfgW8128x128) ? 128 : 256; }
+int gemm_cta_group(int cfg) {
+    return (cfg == kCfgPair256 || cfg == kCfgW8Pair256 || cfg == kCfgAQPair256) ? 2 : 1;
+}
+int gemm_block_m(int cfg) { return 128 * gemm_cta_group(cfg); }
+int gemm_block_n(int cfg) { return (cfg == kCfg128x128 || cfg == kCfgW8128x128 || cfg == kCfgAQ128x128) ? 128 : 256; }
 int gemm_b_box_rows(int cfg) { return cfg == kCfg128x256 ? 256 : 128; }
-int gemm_cta_group(int cfg) { return (cfg == kCfgPair256 || cfg == kCfgW8Pair256) ? 2 : 1; }
 bool gemm_weight_only(int cfg) { return cfg == kCfgW8Pair256 || cfg == kCfgW8128x128; }
+bool gemm_quantizes_a(int cfg) { return cfg == kCfgAQPair256 || cfg == kCfgAQ128x128; }
 int gemm_k_elems(int cfg) { return gemm_weight_only(cfg) ? 64 : 128; }
 
 // MMA units (CTA pairs or CTAs) to launch: one per tile, at most one per SM (pair).
@@ -676,15 +770,19 @@ int gemm_units_for(int cfg, int num_tiles, const DeviceInfo* dev) {
 cudaError_t launch_gemm(int cfg, const GemmArgs& args, int units, cudaStream_t stream) {
     switch (cfg) {
         case kCfgPair256:
-            return launch_cfg<2, 256, false>(args, units, stream);
+            return launch_cfg<2, 256, kOpsFp8>(args, units, stream);
         case kCfg128x256:
-            return launch_cfg<1, 256, false>(args, units, stream);
+            return launch_cfg<1, 256, kOpsFp8>(args, units, stream);
         case kCfg128x128:
-            return launch_cfg<1, 128, false>(args, units, stream);
+            return launch_cfg<1, 128, kOpsFp8>(args, units, stream);
         case kCfgW8Pair256:
-            return launch_cfg<2, 256, true>(args, units, stream);
+            return launch_cfg<2, 256, kOpsW8>(args, units, stream);
         case kCfgW8128x128:
-            return launch_cfg<1, 128, true>(args, units, stream);
+            return launch_cfg<1, 128, kOpsW8>(args, units, stream);
+        case kCfgAQPair256:
+            return launch_cfg<2, 256, kOpsAQ>(args, units, stream);
+        case kCfgAQ128x128:
+            return launch_cfg<1, 128, kOpsAQ>(args, units, stream);
         default:
             return cudaErrorInvalidValue;
     }

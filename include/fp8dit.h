@@ -213,6 +213,28 @@ fp8dit_status fp8_weight_only_linear(fp8dit_linear h, int64_t M, const uint16_t*
                                      fp8dit_stream_t stream);
 
 /*
+ * FP8 linear from a bf16 activation with the quantisation moved into the GEMM
+ * (the fused variant of "从 BF16 到 FP8", section 三.1: runtime activation
+ * quantisation feeding the FP8 GEMM). The per-token amax needs the whole row
+ * before any element can be quantised, so a pre-pass reads A once and writes
+ * per row the scale S = amax / 448 (1 for an all-zero row) and RN(1 / S) (0
+ * where the exact-division quotient is used); the GEMM then loads bf16 tiles
+ * of A and quantises them to E4M3 in shared memory next to the tensor cores.
+ * The FP8 activation is never written to memory.
+ * Result: the codes are the ones fp8_quantize_rowwise writes, so y equals what
+ * fp8_scaled_linear computes from a_bf16 (bit for bit where both use 256 x 256
+ * pair tiles; otherwise within the accumulation-order difference).
+ *   a_bf16 [M, K] bf16 contiguous, 16-byte aligned;
+ *   scale_scratch DEVICE float[2 * M], 4-byte aligned, caller-owned: the
+ *     per-token scales S (first M) then their reciprocals; written by the call,
+ *     S is left there for the caller;
+ *   y [M, N] bf16 contiguous, 16-byte aligned.
+ * M == 0 is a no-op. Must run on the handle's device.
+ */
+fp8dit_status fp8_scaled_linear_fused(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, float* scale_scratch,
+                                      uint16_t* y, fp8dit_stream_t stream);
+
+/*
  * fp8_scaled_linear from a bf16 activation, for callers that cannot allocate
  * device memory. The pages have no counterpart: this entry exists for code
  * that has no way to hand the library qa / sa scratch, such as a plugin whose
