@@ -41,6 +41,8 @@ import numpy as np  # noqa: E402
 
 METRIC = "fused FP8 linear TFLOP/s (% FP8 peak) at FFN shapes; quantizer GB/s (% HBM)"
 WORKLOAD = "FFN-up 4096x8192x2048 + FFN-down 4096x2048x8192 FP8 linear from bf16 activations"
+E2E_CHUNK_ROWS = 2048  # host-pipeline chunk for the end-to-end measurement
+E2E_SLOTS = 2
 FFN = (("up", 4096, 8192, 2048), ("down", 4096, 2048, 8192))
 FLOPS_PER_STEP = sum(2.0 * M * N * K for _, M, N, K in FFN)
 # Quantiser algorithmic bytes: bf16 read + FP8 write + fp32 scale per row.
@@ -422,16 +424,16 @@ def main():
 
 
 def measure_e2e(fp8, torch, layers, host, dev, args, world):
-    """Same metric through FP8Linear.forward with host buffers: every step copies
-    both activations host->device (pinned) and both outputs device->host."""
+    """Same metric through the host-buffer API (FP8Linear.forward_host ->
+    fp8_scaled_linear_host): every step copies both activations host->device
+    from pinned memory and both outputs device->host, chunk by chunk,
+    overlapped with the kernels and with each other by the library's
+    pipeline; the step ends when the last output row has reached host memory."""
     pinned = {}
     for name, M, N, K in FFN:
         a = torch.from_numpy(np.ascontiguousarray(host[name]["A"]).view(np.int16)).view(torch.bfloat16)
-        pinned[name] = {"A": a.pin_memory(), "y": torch.empty((M, N), dtype=torch.bfloat16).pin_memory(),
-                        "Ad": torch.empty((M, K), dtype=torch.bfloat16, device=dev),
-                        "yd": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
-                        "qa": torch.empty((M, K), dtype=torch.uint8, device=dev),
-                        "sa": torch.empty((M,), dtype=torch.float32, device=dev)}
+        pinned[name] = {"A": a.pin_memory(), "y": torch.empty((M, N), dtype=torch.bfloat16).pin_memory()}
+        layers[name].attach_host_pipeline(chunk_rows=E2E_CHUNK_ROWS, slots=E2E_SLOTS)
     h2d = sum(2 * M * K for _, M, N, K in FFN)
     d2h = sum(2 * M * N for _, M, N, K in FFN)
     stream = torch.cuda.current_stream(dev)
@@ -439,9 +441,7 @@ def measure_e2e(fp8, torch, layers, host, dev, args, world):
     def step():
         for name, *_ in FFN:
             p = pinned[name]
-            p["Ad"].copy_(p["A"], non_blocking=True)
-            layers[name].forward(p["Ad"], y=p["yd"], qa_scratch=p["qa"], sa_scratch=p["sa"])
-            p["y"].copy_(p["yd"], non_blocking=True)
+            layers[name].forward_host(p["A"], y=p["y"])
 
     for _ in range(args.warmup):
         step()
@@ -458,9 +458,12 @@ def measure_e2e(fp8, torch, layers, host, dev, args, world):
     t1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), dev)
+    for name, *_ in FFN:
+        layers[name].detach_host_pipeline()
     return {"value": whole_job_rate(world, FLOPS_PER_STEP, steps, ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "api": "FP8Linear.forward (fp8_scaled_linear) + pinned host copies"}
+            "api": f"FP8Linear.forward_host (fp8_scaled_linear_host: chunks of {E2E_CHUNK_ROWS} rows, "
+                   f"{E2E_SLOTS} slots, copy-in / quantise + GEMM / copy-out overlapped) from pinned host memory"}
 
 
 def time_region(torch, fn, iters, dev, warm=3):

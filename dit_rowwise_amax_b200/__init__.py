@@ -80,6 +80,10 @@ def load_library():
     L.fp8_scaled_linear_noalloc.argtypes = [p, i64, p, p, p]
     L.fp8_weight_only_linear.argtypes = [p, i64, p, p, p]
     L.fp8_scaled_linear_fused.argtypes = [p, i64, p, p, p, p]
+    L.fp8_linear_host_workspace_size.argtypes = [p, i64, i32]
+    L.fp8_linear_host_workspace_size.restype = ctypes.c_size_t
+    L.fp8_linear_set_host_pipeline.argtypes = [p, p, ctypes.c_size_t, i64, i32]
+    L.fp8_scaled_linear_host.argtypes = [p, i64, p, p, p]
     L.fp8_linear_plan.argtypes = [p, i64, i32, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.fp8dit_device_error.argtypes = [p]
     L.fp8dit_selftest_expired_wait.argtypes = [i64, p]
@@ -89,6 +93,7 @@ def load_library():
                  "fp8_quantize_weight_per_tensor",
                  "fp8_linear_create", "fp8_linear_destroy", "fp8_scaled_linear", "fp8_scaled_linear_multi",
                  "fp8_scaled_linear_noalloc", "fp8_weight_only_linear", "fp8_scaled_linear_fused",
+                 "fp8_linear_set_host_pipeline", "fp8_scaled_linear_host",
                  "fp8_linear_plan", "fp8_linear_set_workspace", "fp8dit_device_error",
                  "fp8dit_selftest_expired_wait",
                  "fp8dit_selftest_quotient"):
@@ -359,6 +364,40 @@ class FP8Linear:
             raise ValueError("scale_scratch must be a CUDA float32 tensor of at least 2 * M elements")
         _check(load_library().fp8_scaled_linear_fused(self._h, M, a.data_ptr(), scale_scratch.data_ptr(),
                                                       y.data_ptr(), _stream(a.device)))
+        return y
+
+    def attach_host_pipeline(self, chunk_rows: int = 2048, slots: int = 2) -> torch.Tensor:
+        """Allocate and attach the device workspace of the host-buffer pipeline
+        (forward_host); returns it."""
+        L = load_library()
+        need = int(L.fp8_linear_host_workspace_size(self._h, chunk_rows, slots))
+        if need == 0:
+            raise ValueError("chunk_rows must be > 0 and slots in 2..8")
+        ws = torch.empty((need,), dtype=torch.uint8, device=self.device)
+        _check(L.fp8_linear_set_host_pipeline(self._h, ws.data_ptr(), need, chunk_rows, slots))
+        self.host_workspace = ws  # keep it alive while attached
+        return ws
+
+    def detach_host_pipeline(self) -> None:
+        _check(load_library().fp8_linear_set_host_pipeline(self._h, None, 0, 0, 0))
+        self.host_workspace = None
+
+    def forward_host(self, a: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """The FP8 linear of a HOST bf16 activation into a HOST bf16 output,
+        chunks of rows pipelined through copy-in, quantise + GEMM and copy-out
+        (pinned tensors let the copies overlap). Asynchronous on the current
+        stream: the result is in ``y`` once that stream has been synchronised,
+        and ``a`` must stay unchanged until then."""
+        if a.dtype != torch.bfloat16 or a.dim() != 2 or not a.is_contiguous() or a.is_cuda:
+            raise ValueError("a must be a contiguous host bf16 [M, K] tensor")
+        if a.shape[1] != self.K:
+            raise ValueError(f"a must be [M, {self.K}]")
+        M = a.shape[0]
+        if y is None:
+            y = torch.empty((M, self.N), dtype=torch.bfloat16).pin_memory()
+        if y.dtype != torch.bfloat16 or y.shape != (M, self.N) or not y.is_contiguous() or y.is_cuda:
+            raise ValueError(f"y must be a contiguous host bf16 [{M}, {self.N}] tensor")
+        _check(load_library().fp8_scaled_linear_host(self._h, M, a.data_ptr(), y.data_ptr(), _stream(self.device)))
         return y
 
     def forward_fp8(self, qa: torch.Tensor, sa: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:

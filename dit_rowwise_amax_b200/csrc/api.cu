@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "fp8dit_internal.cuh"
+#include "linear_handle.cuh"
 
 // Per-device error word raised by expired bounded waits.
 __device__ uint32_t g_fp8dit_error_word;
@@ -151,19 +152,6 @@ cudaError_t launch_selftest_wait(cudaStream_t stream, DevErr err) {
 }  // namespace fp8dit
 
 using namespace fp8dit;
-
-// ------------------------------------------------------------- linear handle
-struct fp8dit_linear_s {
-    int64_t N, K;
-    const uint8_t* qw;
-    const float* sw;
-    const uint16_t* bias;
-    int device;
-    int num_sms;
-    CUtensorMap tmB[kNumCfgs];  // weight descriptors, one per tile configuration
-    void* sk_ws;                // caller-owned stream-K workspace (or null)
-    size_t sk_ws_bytes;
-};
 
 // Stream-K flag values: unique per launch in this process, never 0 (the value
 // flags hold after fp8_linear_set_workspace clears them).
@@ -456,6 +444,7 @@ fp8dit_status fp8_linear_set_workspace(fp8dit_linear h, void* workspace, size_t 
 
 fp8dit_status fp8_linear_destroy(fp8dit_linear h) {
     t_last_error[0] = 0;
+    if (h) host_pipe_release(h->pipe);
     delete h;
     return FP8DIT_OK;
 }

@@ -235,6 +235,42 @@ fp8dit_status fp8_scaled_linear_fused(fp8dit_linear h, int64_t M, const uint16_t
                                       uint16_t* y, fp8dit_stream_t stream);
 
 /*
+ * FP8 linear from HOST buffers, with the transfers pipelined around the
+ * kernels (the library's runtime for callers whose activations live in host
+ * memory; the pages have no counterpart). The result is fp8_scaled_linear's
+ * from a bf16 activation, row for row (each row depends only on its own
+ * activation row), computed chunk by chunk.
+ *
+ * fp8_linear_host_workspace_size: DEVICE bytes for `slots` slots of
+ *   `chunk_rows` rows (per slot: bf16 activation, FP8 codes, scales, bf16
+ *   output); 0 for invalid arguments (slots must be 2..8, chunk_rows > 0).
+ * fp8_linear_set_host_pipeline: attach caller-owned DEVICE memory (256-byte
+ *   aligned, at least that size) to the layer, creating two copy streams and
+ *   the slot events on the layer's device; NULL workspace detaches (and frees
+ *   the streams and events). The workspace belongs to this layer only and must
+ *   stay allocated until the work of every call using it has completed.
+ * fp8_scaled_linear_host: y_host [M, N] = the linear of a_host [M, K] (both
+ *   bf16, contiguous, HOST memory; page-locked memory is needed for the
+ *   copies to overlap anything). The M rows go in chunks: host-to-device copy
+ *   (copy-in stream) -> quantise + GEMM (`stream`) -> device-to-host copy
+ *   (copy-out stream), chunks and slots in a ring, so both copy directions and
+ *   the kernels overlap, also with the previous call's copy-out.
+ *   Ordering: `stream` passes the end of this call only once every output row
+ *   is in y_host, so synchronising `stream` (or work queued on it later) sees
+ *   the result. The input copies are ordered only after earlier calls' use of
+ *   the same slots, NOT after other work queued on `stream`: a_host must hold
+ *   the activation when the call is made and stay unchanged, and both host
+ *   buffers stay allocated, until `stream` has passed this call. Calls on one
+ *   handle are serialised by a lock. Errors as fp8_scaled_linear, plus
+ *   FP8DIT_ERR_INVALID_ARG when no pipeline is attached.
+ */
+size_t fp8_linear_host_workspace_size(fp8dit_linear h, int64_t chunk_rows, int32_t slots);
+fp8dit_status fp8_linear_set_host_pipeline(fp8dit_linear h, void* workspace, size_t bytes, int64_t chunk_rows,
+                                           int32_t slots);
+fp8dit_status fp8_scaled_linear_host(fp8dit_linear h, int64_t M, const uint16_t* a_host, uint16_t* y_host,
+                                     fp8dit_stream_t stream);
+
+/*
  * fp8_scaled_linear from a bf16 activation, for callers that cannot allocate
  * device memory. The pages have no counterpart: this entry exists for code
  * that has no way to hand the library qa / sa scratch, such as a plugin whose
