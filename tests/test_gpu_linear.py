@@ -48,21 +48,6 @@ def check_full(y, qa, sa, qw, sw, bias):
     return worst
 
 
-def check_sampled(y, qa, sa, qw, sw, bias, n=20000, extra_rows=(), seed=0):
-    M, N = y.shape
-    rng = np.random.default_rng(seed)
-    ms = rng.integers(0, M, n)
-    ns = rng.integers(0, N, n)
-    for r in extra_rows:  # whole rows (e.g. the ragged last tile)
-        ms = np.concatenate([ms, np.full(N, r)])
-        ns = np.concatenate([ns, np.arange(N)])
-    ref = oracle.linear_at(qa, sa, qw, sw, bias, ms, ns)
-    got = bf16_tensor_to_f64(y)[ms, ns]
-    ok, worst = oracle.tolerance_ok(got, ref)
-    assert ok, f"tolerance exceeded: worst error / bound = {worst:.3f}"
-    return worst
-
-
 def test_tiny_config_full():
     d = synth.tiny()
     layer, qw, sw = make_layer(d["W"], d["bias"])
@@ -71,19 +56,19 @@ def test_tiny_config_full():
 
 
 def test_ffn_up_full_size():
+    """Every one of the 4096 x 8192 outputs against the oracle's exact product."""
     d = synth.ffn_up()
     layer, qw, sw = make_layer(d["W"], d["bias"])
     y, qa, sa = run_bf16(layer, d["A"])
-    check_sampled(y, qa, sa, qw, sw, d["bias"], extra_rows=(0, 4095))
-    check_full(y[:192], qa[:192], sa[:192], qw, sw, d["bias"])
+    check_full(y, qa, sa, qw, sw, d["bias"])
 
 
 def test_ffn_down_full_size():
+    """Every one of the 4096 x 2048 outputs (K = 8192) against the oracle."""
     d = synth.ffn_down()
     layer, qw, sw = make_layer(d["W"], d["bias"])
     y, qa, sa = run_bf16(layer, d["A"])
-    check_sampled(y, qa, sa, qw, sw, d["bias"], extra_rows=(1, 4095))
-    check_full(y[:160], qa[:160], sa[:160], qw, sw, d["bias"])
+    check_full(y, qa, sa, qw, sw, d["bias"])
 
 
 @pytest.mark.parametrize("M", [1, 26, 127, 128, 129, 255, 700])
@@ -146,10 +131,7 @@ def test_multi_equals_single_calls_attention_full_size():
         assert np.array_equal(qa.cpu().numpy(), qao) and np.array_equal(sa.cpu().numpy(), sao)
         for y, ys_ref, (qw, sw, b) in zip(ys, singles, refs):
             assert torch.equal(y.view(torch.int16), ys_ref.view(torch.int16))
-            if M > 1000:
-                check_sampled(y, qao, sao, qw, sw, b, n=8000, extra_rows=(M - 1,))
-            else:
-                check_full(y, qao, sao, qw, sw, b)
+            check_full(y, qao, sao, qw, sw, b)  # all 32760 x 2048 outputs of each projection
 
 
 def test_multi_two_and_four_layers_with_different_n():

@@ -47,9 +47,7 @@ def test_stream_k_parity_and_determinism(M, N, K):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), "stream-K result changed between runs"
     assert not torch.equal(y1.view(torch.int16), y_plain.view(torch.int16)), "no tile was split"
     qa, sa = qa_d.cpu().numpy(), sa_d.cpu().numpy()
-    rng = np.random.default_rng(5)
-    rows = np.unique(np.concatenate([np.arange(48), np.arange(M - 48, M), rng.integers(0, M, 48)]))
-    check_rows(y1, qa, sa, qw, sw, bias, rows)
+    check_rows(y1, qa, sa, qw, sw, bias, np.arange(M))  # every output
     layer.detach_workspace()
     y3 = layer.forward_fp8(qa_d, sa_d)
     torch.cuda.synchronize()
