@@ -1,0 +1,78 @@
+"""Run one kernel of the FP8 linear path a few times on the synthetic workload
+inputs, for profiling it on its own (for example under Nsight Compute):
+
+    python -m dit_rowwise_amax_b200.kernel_cases weight_only_ffn_up --iters 4
+
+Cases (inputs from ``synth``, the same as the benchmark's):
+    quantize_ffn_up, quantize_ffn_down   rowwise E4M3 quantiser on the FFN activations
+    gelu_quantize_ffn_down               GELU -> E4M3 producer on a [4096, 8192] activation
+    gemm_ffn_up, gemm_ffn_down           FP8 GEMM + epilogue from pre-quantised activations
+    weight_only_ffn_up, ..._ffn_down     FP8 weight-only GEMM (bf16 activation)
+    fused_ffn_up, fused_ffn_down         quantise-in-GEMM variant (row-scale pre-pass + GEMM)
+Layer creation runs the per-channel weight quantiser first; every case then
+launches only its own kernels. Exits non-zero if the device reports an error.
+"""
+import argparse
+import sys
+
+import numpy as np
+import torch
+
+import synth
+
+from . import FP8Linear, act_quantize_rowwise, device_error, quantize_rowwise
+
+CASES = ("quantize_ffn_up", "quantize_ffn_down", "gelu_quantize_ffn_down", "gemm_ffn_up", "gemm_ffn_down",
+         "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down")
+
+
+def _dev(a: np.ndarray, dev) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def run(case: str, iters: int) -> None:
+    dev = torch.device("cuda", 0)
+    workload = synth.ffn_up() if case.endswith("ffn_up") else synth.ffn_down()
+    a = _dev(workload["A"], dev)
+    M, K = a.shape
+    if case.startswith("quantize"):
+        q = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        s = torch.empty((M,), dtype=torch.float32, device=dev)
+        for _ in range(iters):
+            quantize_rowwise(a, q=q, scale=s)
+    elif case.startswith("gelu_quantize"):
+        q = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        s = torch.empty((M,), dtype=torch.float32, device=dev)
+        for _ in range(iters):
+            act_quantize_rowwise(a, "gelu", q=q, scale=s)
+    else:
+        layer = FP8Linear.from_weight(_dev(workload["W"], dev), _dev(workload["bias"], dev))
+        y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=dev)
+        if case.startswith("gemm"):
+            qa, sa = quantize_rowwise(a)
+            for _ in range(iters):
+                layer.forward_fp8(qa, sa, y=y)
+        elif case.startswith("weight_only"):
+            for _ in range(iters):
+                layer.forward_weight_only(a, y=y)
+        else:
+            sc = torch.empty((2 * M,), dtype=torch.float32, device=dev)
+            for _ in range(iters):
+                layer.forward_fused(a, y=y, scale_scratch=sc)
+    torch.cuda.synchronize()
+    if device_error() != 0:
+        raise SystemExit(f"{case}: device error word set")
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("case", choices=CASES)
+    ap.add_argument("--iters", type=int, default=4)
+    args = ap.parse_args(argv)
+    run(args.case, args.iters)
+    print("ok", args.case)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
