@@ -153,17 +153,6 @@ cudaError_t launch_selftest_wait(cudaStream_t stream, DevErr err) {
 
 using namespace fp8dit;
 
-// Stream-K flag values: unique per launch in this process, never 0 (the value
-// flags hold after fp8_linear_set_workspace clears them).
-static std::atomic<uint32_t> g_sk_epoch{0};
-static uint32_t next_sk_epoch() {
-    uint32_t e;
-    do {
-        e = g_sk_epoch.fetch_add(1) + 1;
-    } while (e == 0);
-    return e;
-}
-
 int64_t fp8dit::linear_k(const fp8dit_linear_s* h) { return h->K; }
 
 static int64_t tiles_for(const fp8dit_linear_s* h, int64_t M, int n_problems, int cfg) {
@@ -250,7 +239,6 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
         const int64_t waves = (tiles + units - 1) / units;
         if ((waves * units - tiles) * 4 > waves * units) {
             args.stream_k = 1;
-            args.sk_epoch = next_sk_epoch();
             args.sk_flag = static_cast<uint32_t*>(hs[0]->sk_ws);
             args.sk_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(hs[0]->sk_ws) +
                                                        (stream_k_workspace_bytes(units) -

@@ -101,9 +101,9 @@ struct alignas(64) GemmArgs {
     // Stream-K schedule (pair FP8 configuration only): each MMA unit takes an
     // equal contiguous share of the num_tiles x num_kb k-blocks. A tile split
     // between units u and u+1 is finished by u: u+1 computes its k-block tail
-    // first, stores the fp32 partial in sk_partial and publishes sk_flag.
+    // first, stores the fp32 partial in sk_partial and sets sk_flag to 1; u
+    // waits for 1, adds the partial and clears the flag again.
     int32_t stream_k;
-    uint32_t sk_epoch;   // flag value that marks this launch's partials
     uint32_t* sk_flag;   // [units][2 CTAs][8 epilogue warps]
     float* sk_partial;   // [units][2 CTAs][8 epilogue warps][32 rows][128 columns]
 };

@@ -453,10 +453,10 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 // before this unit's last one; wait, bounded, for its flag, then
                 // fetch the first chunk while the accumulator is still being built.
                 const uint32_t* flag = args.sk_flag + ((size_t)(unit + 1) * 2 + rank) * C::EPI_WARPS + ew;
-                bool ok = ld_acquire_gpu_u32(flag) == args.sk_epoch;
+                bool ok = ld_acquire_gpu_u32(flag) == 1u;
                 if (!ok) {
                     const unsigned long long t0 = globaltimer_ns();
-                    while (!(ok = ld_acquire_gpu_u32(flag) == args.sk_epoch)) {
+                    while (!(ok = ld_acquire_gpu_u32(flag) == 1u)) {
                         if (*abort_flag) break;
                         if (globaltimer_ns() - t0 > args.err.limit_ns) {
                             *abort_flag = 1;
@@ -551,7 +551,14 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 __threadfence();
                 __syncwarp();
                 if (lane == 0)
-                    st_release_gpu_u32(args.sk_flag + ((size_t)unit * 2 + rank) * C::EPI_WARPS + ew, args.sk_epoch);
+                    st_release_gpu_u32(args.sk_flag + ((size_t)unit * 2 + rank) * C::EPI_WARPS + ew, 1u);
+            }
+            if (head) {
+                // Every lane has its partial in registers: clear the flag, so the
+                // workspace is ready for the next launch without a host reset
+                // (stream-ordered launches, CUDA graph replays included).
+                __syncwarp();
+                if (lane == 0) args.sk_flag[((size_t)(unit + 1) * 2 + rank) * C::EPI_WARPS + ew] = 0u;
             }
             tc_fence_before();
             __syncwarp();

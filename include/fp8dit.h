@@ -177,9 +177,13 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  *     148 SMs), the same for every M.
  *   fp8_linear_set_workspace: attach caller-owned DEVICE memory (256-byte
  *     aligned, at least that size) or detach with NULL. Attaching clears the
- *     workspace's flags (synchronously). The workspace may be attached to
- *     several layers whose calls run one after another on the GPU; calls that
- *     overlap on the GPU must not share a workspace.
+ *     workspace's flags (synchronously); every launch leaves them cleared, so
+ *     stream-ordered launches and replays of a captured CUDA graph need no
+ *     host reset. After a call whose device error word reports
+ *     FP8DIT_ERR_TIMEOUT, attach the workspace again before reusing it. The
+ *     workspace may be attached to several layers whose calls run one after
+ *     another on the GPU; calls that overlap on the GPU must not share a
+ *     workspace.
  */
 size_t fp8_linear_workspace_size(fp8dit_linear h);
 fp8dit_status fp8_linear_set_workspace(fp8dit_linear h, void* workspace, size_t bytes);

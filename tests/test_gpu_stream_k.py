@@ -78,3 +78,36 @@ def test_ffn_shapes_keep_plain_schedule():
     y_ws = layer.forward_fp8(qa_d, sa_d)
     torch.cuda.synchronize()
     assert torch.equal(y_ws.view(torch.int16), y_plain.view(torch.int16))
+
+
+def test_stream_k_cuda_graph_replays():
+    """Stream-K launches replayed from a captured CUDA graph: every launch
+    leaves the workspace flags cleared, so each replay (with new inputs copied
+    into the captured buffers) equals the eager result for those inputs."""
+    M, N, K = 4800, 2048, 1040  # 152 pair tiles: the split schedule
+    W = synth.normal_bf16(f"gpu/sk/W/{N}x{K}", (N, K), 0.02)
+    layer, _, _ = layer_and_codes(W, synth.normal_bf16(f"gpu/sk/b/{N}", (N,), 0.1))
+    layer.attach_workspace()
+    inputs = [fp8.quantize_rowwise(to_device_bf16(synth.normal_bf16(f"gpu/sk/graph/A{i}", (M, K), 1.0)))
+              for i in range(3)]
+    eager = [layer.forward_fp8(qa, sa) for qa, sa in inputs]
+    torch.cuda.synchronize()
+    qa_buf, sa_buf = inputs[0][0].clone(), inputs[0][1].clone()
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        layer.forward_fp8(qa_buf, sa_buf, y=y)  # warm-up on the capture stream
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward_fp8(qa_buf, sa_buf, y=y)
+    for rep in range(2):
+        for (qa, sa), ref in zip(inputs, eager):
+            qa_buf.copy_(qa)
+            sa_buf.copy_(sa)
+            g.replay()
+            torch.cuda.synchronize()
+            assert fp8.device_error() == 0
+            assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), f"replay {rep} differs"
