@@ -9,6 +9,7 @@ Cases (inputs from ``synth``, the same as the benchmark's):
     gemm_ffn_up, gemm_ffn_down           FP8 GEMM + epilogue from pre-quantised activations
     weight_only_ffn_up, ..._ffn_down     FP8 weight-only GEMM (bf16 activation)
     fused_ffn_up, fused_ffn_down         quantise-in-GEMM variant (row-scale pre-pass + GEMM)
+    state_dict_e4m3fn, state_dict_e5m2   per-tensor conversion of the 192-tensor DiT weight set
 Layer creation runs the per-channel weight quantiser first; every case then
 launches only its own kernels. Exits non-zero if the device reports an error.
 """
@@ -20,10 +21,11 @@ import torch
 
 import synth
 
-from . import FP8Linear, act_quantize_rowwise, device_error, quantize_rowwise
+from . import E4M3FN, E5M2, FP8Linear, act_quantize_rowwise, device_error, quantize_per_tensor, quantize_rowwise
 
 CASES = ("quantize_ffn_up", "quantize_ffn_down", "gelu_quantize_ffn_down", "gemm_ffn_up", "gemm_ffn_down",
-         "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down")
+         "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down", "state_dict_e4m3fn",
+         "state_dict_e5m2")
 
 
 def _dev(a: np.ndarray, dev) -> torch.Tensor:
@@ -32,6 +34,17 @@ def _dev(a: np.ndarray, dev) -> torch.Tensor:
 
 def run(case: str, iters: int) -> None:
     dev = torch.device("cuda", 0)
+    if case.startswith("state_dict"):
+        tensors = [_dev(synth.state_dict_tensor(n, s), dev) for n, s in synth.state_dict_layout()]
+        outs = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in tensors]
+        scales = torch.empty((len(tensors),), dtype=torch.float32, device=dev)
+        fmt = E4M3FN if case.endswith("e4m3fn") else E5M2
+        for _ in range(iters):
+            quantize_per_tensor(tensors, fmt, outs=outs, scales=scales)
+        torch.cuda.synchronize()
+        if device_error() != 0:
+            raise SystemExit(f"{case}: device error word set")
+        return
     workload = synth.ffn_up() if case.endswith("ffn_up") else synth.ffn_down()
     a = _dev(workload["A"], dev)
     M, K = a.shape
