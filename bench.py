@@ -41,6 +41,7 @@ import numpy as np  # noqa: E402
 
 METRIC = "fused FP8 linear TFLOP/s (% FP8 peak) at FFN shapes; quantizer GB/s (% HBM)"
 WORKLOAD = "FFN-up 4096x8192x2048 + FFN-down 4096x2048x8192 FP8 linear from bf16 activations"
+REFERENCE_BUDGET_S = 120.0  # whole --impl reference run, seconds
 E2E_CHUNK_ROWS = 2048  # host-pipeline chunk for the end-to-end measurement
 E2E_SLOTS = 2
 FFN = (("up", 4096, 8192, 2048), ("down", 4096, 2048, 8192))
@@ -234,7 +235,10 @@ def run_reference(args, world, rank):
         return
     import oracle
     data = oracle_data()
-    rows = calibrate_rows(data, 1.5)
+    # Each step is sized so that the whole run (warm-up included) takes about
+    # REFERENCE_BUDGET_S, and at most 1.5 s a step.
+    per_step_s = min(1.5, REFERENCE_BUDGET_S / (args.steps + args.warmup))
+    rows = calibrate_rows(data, per_step_s)
     for _ in range(args.warmup):
         oracle_sample_step(data, rows)
     t0 = time.perf_counter()
