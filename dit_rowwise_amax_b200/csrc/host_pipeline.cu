@@ -62,7 +62,13 @@ void host_pipe_release(HostPipe* p) {
     int prev = 0;
     const bool switched = cudaGetDevice(&prev) == cudaSuccess && prev != p->device &&
                           cudaSetDevice(p->device) == cudaSuccess;
-    // Streams and events with pending work are released once that work ends.
+    // Wait for the pipeline's work in flight (the last compute and copy-out
+    // of every slot used), so that the workspace is free when this returns.
+    for (int s = 0; s < p->slots; ++s) {
+        if (!p->used[s]) continue;
+        cudaEventSynchronize(p->comp_done[s]);
+        cudaEventSynchronize(p->out_done[s]);
+    }
     for (int s = 0; s < kMaxSlots; ++s) {
         if (p->in_done[s]) cudaEventDestroy(p->in_done[s]);
         if (p->comp_done[s]) cudaEventDestroy(p->comp_done[s]);

@@ -176,8 +176,9 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  *   fp8_linear_workspace_size: bytes needed on the layer's device (~19 MB on
  *     148 SMs), the same for every M.
  *   fp8_linear_set_workspace: attach caller-owned DEVICE memory (256-byte
- *     aligned, at least that size) or detach with NULL. Attaching clears the
- *     workspace's flags (synchronously); every launch leaves them cleared, so
+ *     aligned, at least that size) or detach with NULL, while no call that
+ *     uses the layer is in flight. Attaching clears the workspace's flags
+ *     (synchronously); every launch leaves them cleared, so
  *     stream-ordered launches and replays of a captured CUDA graph need no
  *     host reset. After a call whose device error word reports
  *     FP8DIT_ERR_TIMEOUT, attach the workspace again before reusing it. The
@@ -251,8 +252,10 @@ fp8dit_status fp8_scaled_linear_fused(fp8dit_linear h, int64_t M, const uint16_t
  * fp8_linear_set_host_pipeline: attach caller-owned DEVICE memory (256-byte
  *   aligned, at least that size) to the layer, creating two copy streams and
  *   the slot events on the layer's device; NULL workspace detaches (and frees
- *   the streams and events). The workspace belongs to this layer only and must
- *   stay allocated until the work of every call using it has completed.
+ *   the streams and events). Replacing or detaching a pipeline, and
+ *   fp8_linear_destroy, first wait on the host for that pipeline's work in
+ *   flight. The workspace belongs to this layer only and must stay allocated
+ *   until the work of every call using it has completed.
  * fp8_scaled_linear_host: y_host [M, N] = the linear of a_host [M, K] (both
  *   bf16, contiguous, HOST memory; page-locked memory is needed for the
  *   copies to overlap anything). The M rows go in chunks: host-to-device copy

@@ -120,3 +120,22 @@ def test_argument_errors():
     assert L.fp8_linear_set_host_pipeline(h, None, 0, 0, 0) == 0  # detach
     assert L.fp8_scaled_linear_host(h, 16, a.data_ptr(), y.data_ptr(), s) == 1
     assert fp8.device_error() == 0
+
+
+def test_reattach_while_work_in_flight():
+    """Re-attaching a pipeline to the same workspace while a call is still
+    queued waits for that call's work, so neither result is corrupted."""
+    M, N, K = 2048, 512, 1024
+    W = synth.normal_bf16("gpu/host/re/W", (N, K), 0.02)
+    layer, _, _ = make_layer(W, None)
+    ws = layer.attach_host_pipeline(chunk_rows=256, slots=2)
+    L = fp8.load_library()
+    A0 = synth.normal_bf16("gpu/host/re/A0", (M, K), 1.0)
+    A1 = synth.normal_bf16("gpu/host/re/A1", (M, K), 1.0)
+    a0, a1 = host_bf16(A0), host_bf16(A1)
+    y0 = layer.forward_host(a0)                 # queued, not synchronised
+    assert L.fp8_linear_set_host_pipeline(layer.handle, ws.data_ptr(), ws.numel(), 256, 2) == 0
+    y1 = layer.forward_host(a1)
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), device_reference(layer, A0, 256).view(torch.int16))
+    assert torch.equal(y1.view(torch.int16), device_reference(layer, A1, 256).view(torch.int16))
