@@ -127,3 +127,15 @@ def test_argument_errors_launch_nothing():
     assert L.fp8_scaled_linear_fused(None, 16, a.data_ptr(), sc.data_ptr(), y.data_ptr(), s) == 1
     torch.cuda.synchronize()
     assert fp8.device_error() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 264, 16384), (37, 24, 8208)])
+def test_long_rows_two_pass_scale_prepass(M, N, K):
+    """Rows longer than 8192 elements take the two-pass row-scale pre-pass
+    (scales only, no codes written)."""
+    A = synth.normal_bf16(f"gpu/fused/long/A/{M}x{K}", (M, K), 1.0, outlier_p=0.01, outlier_factor=20.0)
+    W = synth.normal_bf16(f"gpu/fused/long/W/{N}x{K}", (N, K), 0.02)
+    bias = synth.normal_bf16(f"gpu/fused/long/b/{N}", (N,), 0.1)
+    layer, qw, sw = make_layer(W, bias)
+    y, qa, sa = run_fused(layer, A)
+    check_rows(y, qa, sa, qw, sw, bias, np.arange(M))
