@@ -39,6 +39,15 @@
  *    fp8dit_device_error() reads and clears it.
  *  - On any status other than FP8DIT_OK, fp8dit_last_error_string() (per
  *    thread) describes the failure.
+ *  - CUDA graphs: the quantisers, the linear entry points (single, multi,
+ *    weight-only, fused, stream-K) and the per-tensor conversion only enqueue
+ *    kernels (and, per-tensor, a memset), so they can be captured into a
+ *    graph and replayed; each replay reads whatever the captured buffers hold
+ *    then. Make the first fp8_act_quantize_rowwise call on a device (it builds
+ *    its activation tables and synchronises once) and the first
+ *    fp8_scaled_linear_noalloc call on a device before capturing.
+ *    fp8_scaled_linear_host uses its own copy streams and is not meant for
+ *    capture.
  */
 #ifndef FP8DIT_H
 #define FP8DIT_H
