@@ -188,7 +188,8 @@ static int choose_cfg_fused(const fp8dit_linear_s* h, int64_t M) {
 }
 
 // a: FP8 codes [M, K] (qa) for the FP8 x FP8 configurations, bf16 [M, K] for
-// the weight-only ones; sa: per-token scales, or NULL (weight-only).
+// the weight-only and quantise-in-GEMM ones; sa: per-token scales, or NULL
+// (weight-only); ra: the per-token reciprocals (quantise-in-GEMM only).
 static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, const void* a, const float* sa,
                               uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev, int cfg,
                               const float* ra = nullptr) {
@@ -211,7 +212,11 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
             : encode_tma_2d(&args.tmA, 1, a, (uint64_t)K, (uint64_t)M, (uint64_t)K, (uint32_t)ke, 128,
                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != FP8DIT_OK) return st;
-    const int tiles_m = (int)((M + bm - 1) / bm);
+    const int64_t tiles_m64 = (M + bm - 1) / bm;
+    int64_t tiles64 = 0;
+    for (int g = 0; g < n; ++g) tiles64 += tiles_m64 * ((hs[g]->N + bn - 1) / bn);
+    if (tiles64 > INT32_MAX) return unsupported("more than 2^31 - 1 output tiles");
+    const int tiles_m = (int)tiles_m64;
     int tiles = 0;
     for (int g = 0; g < n; ++g) {
         args.tmB[g] = hs[g]->tmB[cfg];
@@ -230,7 +235,8 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
     // launch would keep its units busy for less than 3/4 of its waves (a nearly
     // empty last wave), with at least kSkMinKBlocks k-blocks per tile.
     // Measured on B200: 150 to 152 tiles on 74 pairs (3 waves, 68% busy) run
-    // 13-18% faster split; 128 tiles (2 waves, 86% busy) run 6% slower, since
+    // 2-18% faster split, depending on the power state; 128 tiles (2 waves,
+    // 86% busy) run 6% slower, since
     // under the power cap the SMs left idle in a data-parallel last wave let
     // the busy ones clock higher, which recovers most of the idle time.
     const int units = gemm_units_for(cfg, tiles, dev);
