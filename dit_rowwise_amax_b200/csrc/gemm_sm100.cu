@@ -14,8 +14,9 @@
 //   warp 1      allocates TMEM; one thread of the pair's leader CTA issues
 //               tcgen05.mma (K = 32 per instruction) into a TMEM accumulator
 //               and commits each ring slot back to the producers;
-//   warps 2..9  epilogue, two warps per TMEM lane quarter, each taking half
-//               of the tile's columns: fetch the next tile's sw / bias / sa
+//   warps 2..9  epilogue (kOpsFp8; four warps, one per lane quarter, in the
+//               converter modes), two warps per TMEM lane quarter, each taking
+//               half of the tile's columns: fetch the next tile's sw / bias / sa
 //               while this tile is processed, tcgen05.ld 32 accumulator
 //               columns at a time, scale, bias, bf16, write a 32 x 32 box
 //               into the warp's 64-byte-swizzled staging buffer and
@@ -29,6 +30,18 @@
 // Per-SM shared-memory traffic per MMA is half that of a 1-CTA tile, which
 // lets a 6-deep ring of 32 KB stages cover the L2 latency. No TMA load
 // anywhere uses multicast.
+//
+// Operand modes (OPS): kOpsFp8 is the FP8 linear above. kOpsW8 (FP8
+// weight-only: bf16 A x E4M3 W, "longcat-avatar-compare", section 速度总览)
+// and kOpsAQ (bf16 A quantised per token inside the GEMM) add one converter
+// warp per ring stage after the epilogue warps, which turns the stage's W codes
+// into bf16 (W8) or its bf16 A tile into E4M3 codes (AQ) in place in shared
+// memory before releasing the stage to the MMA.
+//
+// Schedules: data-parallel (tile t on MMA unit t mod units) or, with a
+// workspace, stream-K (each unit an equal share of all k-blocks; a tile split
+// between two units is finished by one of them after the other has published
+// its fp32 partial), see SegSched.
 //
 // Every mbarrier wait is bounded (mbar_wait_bounded): on expiry the CTA
 // raises the device error word and its own and its peer's abort flags, lets
