@@ -217,6 +217,35 @@ def calibrate_rows(data, target_s: float) -> int:
     return int(max(probe, min(4096, probe * target_s / dt)))
 
 
+def oracle_component_rates(data, rows: int) -> dict:
+    """The oracle's parts timed on their own: the exact GEMM per FFN layer on
+    all cores, and the quantisers single-threaded and on all cores (GB/s of
+    bf16 read + codes written + scales)."""
+    import oracle
+    import synth
+    out = {"gemm_gflops_all_cores": {}, "rowwise_quantiser_gbs": {}, "per_tensor_quantiser_gbs": {}}
+    for name, M, N, K in FFN:
+        d = data[name]
+        qa, sa = oracle.quantize_rows(d["A"][:rows], oracle.E4M3FN)
+        t0 = time.perf_counter()
+        oracle.linear(qa, sa, d["qw"], d["sw"], d["bias"])
+        out["gemm_gflops_all_cores"][f"ffn_{name}"] = 2.0 * rows * N * K / (time.perf_counter() - t0) / 1e9
+    hidden = synth.attention()["hidden"][:4096]
+    tensor = synth.state_dict_tensor(*synth.state_dict_layout()[4])  # a [8192, 2048] FFN weight
+    for threads, label in ((1, "1_thread"), (0, f"{oracle.num_threads()}_threads")):
+        oracle.set_threads(threads)
+        t0 = time.perf_counter()
+        oracle.quantize_rows(hidden, oracle.E4M3FN)
+        out["rowwise_quantiser_gbs"][label] = (3 * hidden.size + 4 * hidden.shape[0]) / (time.perf_counter() - t0) / 1e9
+        t0 = time.perf_counter()
+        oracle.quantize_tensor(tensor, oracle.E4M3FN)
+        out["per_tensor_quantiser_gbs"][label] = (3 * tensor.size + 4) / (time.perf_counter() - t0) / 1e9
+    oracle.set_threads(0)
+    out["samples"] = (f"GEMM: first {rows} rows of each FFN layer; rowwise: hidden_states rows 0..4095 "
+                      f"[4096, 2048]; per-tensor: one [8192, 2048] weight")
+    return out
+
+
 def cpu_baseline(target_s: float = 12.0) -> dict:
     import oracle
     data = oracle_data()
@@ -226,7 +255,7 @@ def cpu_baseline(target_s: float = 12.0) -> dict:
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"first {rows} rows of both FFN linears (quantise + exact GEMM + epilogue), {dt:.1f} s",
-            "cpu": cpu_model()}
+            "cpu": cpu_model(), "components": oracle_component_rates(data, max(16, rows // 4))}
 
 
 def run_reference(args, world, rank):

@@ -75,6 +75,8 @@ def _load():
         lib.or_act_bf16.argtypes = [ctypes.c_int, _p, _i64, _p]
         lib.or_num_threads.restype = ctypes.c_int
         lib.or_num_threads.argtypes = []
+        lib.or_set_threads.restype = None
+        lib.or_set_threads.argtypes = [ctypes.c_int]
         lib.or_dot_units.restype = None
         lib.or_dot_units.argtypes = [_p, _p, _i64, _i64, _i64, _p]
         _lib = lib
@@ -198,6 +200,11 @@ def act_bf16(kind: int, h: np.ndarray) -> np.ndarray:
 def num_threads() -> int:
     """Threads the oracle's OpenMP loops use."""
     return int(_load().or_num_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads for the oracle's loops from now on; n <= 0 restores the default."""
+    _load().or_set_threads(int(n))
 
 
 def tolerance_ok(gpu: np.ndarray, ref: np.ndarray, rms_ref: float | None = None):

@@ -299,3 +299,11 @@ void or_encode_many(int fmt, const float* v, int64_t n, uint8_t* out) {
 
 /* Threads the oracle's parallel loops use (for reports). */
 int or_num_threads(void) { return omp_get_max_threads(); }
+
+/* Threads for the parallel loops that follow (timing the oracle single-threaded
+   and on all cores); n <= 0 restores the default. */
+void or_set_threads(int n) {
+    static int default_threads = 0;
+    if (default_threads == 0) default_threads = omp_get_max_threads();
+    omp_set_num_threads(n > 0 ? n : default_threads);
+}
