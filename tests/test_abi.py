@@ -49,3 +49,16 @@ def test_built_for_sm100a_only():
     flags = " ".join(build.NVCC_FLAGS)
     assert "arch=compute_100a,code=sm_100a" in flags
     assert "use_fast_math" not in flags
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/fp8dit.h in a C11 translation unit (the plain-C caller used by
+    the GPU tests), compiled without linking."""
+    import shutil
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    if shutil.which("gcc") is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime.h")):
+        pytest.skip("needs gcc and the CUDA headers")
+    r = subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-c", os.path.join(ROOT, "tests", "c_abi_harness.c"),
+                        "-I" + os.path.join(ROOT, "include"), "-I" + cuda_inc, "-o", str(tmp_path / "h.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
