@@ -129,6 +129,28 @@ def _bf16_matrix(x: torch.Tensor, name: str) -> torch.Tensor:
     return x
 
 
+_CODE_DTYPES = (torch.uint8, torch.float8_e4m3fn, torch.float8_e5m2)
+_BF16_DTYPES = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def _check_out(t: torch.Tensor, name: str, dtypes, shape, device: torch.device, rows_only: bool = False):
+    """A caller-supplied output or scratch tensor: the library writes through
+    its data pointer, so dtype, shape and device must be exactly right.
+    rows_only: only the last dimension needs to be contiguous (row stride free)."""
+    ok = (isinstance(t, torch.Tensor) and t.dtype in dtypes and tuple(t.shape) == tuple(shape)
+          and t.device == device and (t.stride(-1) == 1 if rows_only else t.is_contiguous()))
+    if not ok:
+        names = "/".join(str(d).replace("torch.", "") for d in dtypes)
+        raise ValueError(f"{name} must be a {'row-contiguous' if rows_only else 'contiguous'} {names} tensor "
+                         f"of shape {tuple(shape)} on {device}")
+    return t
+
+
+def _same_device(t: torch.Tensor, device: torch.device, name: str):
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the layer on {device}")
+
+
 def as_float8(q: torch.Tensor, fmt=E4M3FN) -> torch.Tensor:
     """View raw FP8 codes (uint8) as torch's float8 dtype of the format."""
     return q.view(_TORCH_FP8[_fmt(fmt)])
@@ -143,6 +165,8 @@ def quantize_rowwise(x: torch.Tensor, fmt=E4M3FN, q: Optional[torch.Tensor] = No
         q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     if scale is None:
         scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check_out(q, "q", _CODE_DTYPES, (M, K), x.device, rows_only=True)
+    _check_out(scale, "scale", (torch.float32,), (M,), x.device)
     _check(load_library().fp8_quantize_rowwise(x.data_ptr(), M, K, x.stride(0), _fmt(fmt), q.data_ptr(),
                                                q.stride(0), scale.data_ptr(), _stream(x.device)))
     return q, scale
@@ -161,6 +185,8 @@ def act_quantize_rowwise(h: torch.Tensor, act: str = "gelu", q: Optional[torch.T
         q = torch.empty((M, K), dtype=torch.uint8, device=h.device)
     if scale is None:
         scale = torch.empty((M,), dtype=torch.float32, device=h.device)
+    _check_out(q, "q", _CODE_DTYPES, (M, K), h.device, rows_only=True)
+    _check_out(scale, "scale", (torch.float32,), (M,), h.device)
     g = torch.empty((M, K), dtype=torch.bfloat16, device=h.device) if return_bf16 else None
     try:
         kind = ACTIVATIONS[act]
@@ -204,15 +230,22 @@ def quantize_per_tensor(tensors: Sequence[torch.Tensor], fmt=E5M2,
         outs = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in tensors]
     if scales is None:
         scales = torch.ones((n,), dtype=torch.float32, device=dev)
+    if len(outs) != n:
+        raise ValueError("outs must hold one tensor per input tensor")
+    for i, (t, o) in enumerate(zip(tensors, outs)):
+        _check_out(o, f"outs[{i}]", _CODE_DTYPES, t.shape, dev)
+    _check_out(scales, "scales", (torch.float32,), (n,), dev)
     ws_bytes = int(L.fp8_quantize_weight_per_tensor_workspace_size(n))
     if workspace is None:
         workspace = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    if workspace.device != dev or not workspace.is_contiguous() or workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError(f"workspace must be a contiguous tensor of at least {ws_bytes} bytes on {dev}")
     descs = (_TensorDesc * n)()
     for i, (t, o) in enumerate(zip(tensors, outs)):
         descs[i].src, descs[i].numel, descs[i].dst = t.data_ptr(), t.numel(), o.data_ptr()
         descs[i].scale = scales.data_ptr() + 4 * i
-    _check(L.fp8_quantize_weight_per_tensor(descs, n, _fmt(fmt), workspace.data_ptr(), workspace.numel(),
-                                            _stream(dev)))
+    _check(L.fp8_quantize_weight_per_tensor(descs, n, _fmt(fmt), workspace.data_ptr(),
+                                            workspace.numel() * workspace.element_size(), _stream(dev)))
     return list(outs), scales
 
 
@@ -322,12 +355,16 @@ class FP8Linear:
         if not a.is_contiguous() or a.shape[1] != self.K:
             raise ValueError(f"a must be contiguous [M, {self.K}]")
         M = a.shape[0]
+        _same_device(a, self.device, "a")
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.bfloat16, device=a.device)
         if qa_scratch is None:
             qa_scratch = torch.empty((M, self.K), dtype=torch.uint8, device=a.device)
         if sa_scratch is None:
             sa_scratch = torch.empty((M,), dtype=torch.float32, device=a.device)
+        _check_out(y, "y", _BF16_DTYPES, (M, self.N), a.device)
+        _check_out(qa_scratch, "qa_scratch", _CODE_DTYPES, (M, self.K), a.device)
+        _check_out(sa_scratch, "sa_scratch", (torch.float32,), (M,), a.device)
         _check(load_library().fp8_scaled_linear(self._h, M, a.data_ptr(), None, None, qa_scratch.data_ptr(),
                                                 sa_scratch.data_ptr(), y.data_ptr(), _stream(a.device)))
         return y
@@ -341,8 +378,10 @@ class FP8Linear:
         if not a.is_contiguous() or a.shape[1] != self.K:
             raise ValueError(f"a must be contiguous [M, {self.K}]")
         M = a.shape[0]
+        _same_device(a, self.device, "a")
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.bfloat16, device=a.device)
+        _check_out(y, "y", _BF16_DTYPES, (M, self.N), a.device)
         _check(load_library().fp8_weight_only_linear(self._h, M, a.data_ptr(), y.data_ptr(), _stream(a.device)))
         return y
 
@@ -356,12 +395,13 @@ class FP8Linear:
         if not a.is_contiguous() or a.shape[1] != self.K:
             raise ValueError(f"a must be contiguous [M, {self.K}]")
         M = a.shape[0]
+        _same_device(a, self.device, "a")
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.bfloat16, device=a.device)
         if scale_scratch is None:
             scale_scratch = torch.empty((2 * M,), dtype=torch.float32, device=a.device)
-        if scale_scratch.dtype != torch.float32 or scale_scratch.numel() < 2 * M or not scale_scratch.is_cuda:
-            raise ValueError("scale_scratch must be a CUDA float32 tensor of at least 2 * M elements")
+        _check_out(y, "y", _BF16_DTYPES, (M, self.N), a.device)
+        _check_out(scale_scratch, "scale_scratch", (torch.float32,), (2 * M,), a.device)
         _check(load_library().fp8_scaled_linear_fused(self._h, M, a.data_ptr(), scale_scratch.data_ptr(),
                                                       y.data_ptr(), _stream(a.device)))
         return y
@@ -406,8 +446,13 @@ class FP8Linear:
         if qa.shape[1] != self.K or sa.dtype != torch.float32 or sa.shape != (qa.shape[0],):
             raise ValueError("qa [M, K] and sa float32 [M] must match the layer")
         M = qa.shape[0]
+        _same_device(qa, self.device, "qa")
+        _same_device(sa, self.device, "sa")
+        if not sa.is_contiguous():
+            raise ValueError("sa must be contiguous")
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.bfloat16, device=qa.device)
+        _check_out(y, "y", _BF16_DTYPES, (M, self.N), qa.device)
         _check(load_library().fp8_scaled_linear(self._h, M, None, qa.data_ptr(), sa.data_ptr(), None, None,
                                                 y.data_ptr(), _stream(qa.device)))
         return y
@@ -422,12 +467,24 @@ def scaled_linear_multi(layers: Sequence[FP8Linear], a: torch.Tensor,
     a = _bf16_matrix(a, "a")
     n = len(layers)
     M, K = a.shape
+    if not a.is_contiguous():
+        raise ValueError("a must be contiguous")
+    for i, l in enumerate(layers):
+        if l.K != K:
+            raise ValueError(f"layers[{i}] has K = {l.K}, the activation {K}")
+        _same_device(a, l.device, "a")
     if ys is None:
         ys = [torch.empty((M, l.N), dtype=torch.bfloat16, device=a.device) for l in layers]
     if qa_scratch is None:
         qa_scratch = torch.empty((M, K), dtype=torch.uint8, device=a.device)
     if sa_scratch is None:
         sa_scratch = torch.empty((M,), dtype=torch.float32, device=a.device)
+    if len(ys) != n:
+        raise ValueError("ys must hold one output per layer")
+    for i, (y, l) in enumerate(zip(ys, layers)):
+        _check_out(y, f"ys[{i}]", _BF16_DTYPES, (M, l.N), a.device)
+    _check_out(qa_scratch, "qa_scratch", _CODE_DTYPES, (M, K), a.device)
+    _check_out(sa_scratch, "sa_scratch", (torch.float32,), (M,), a.device)
     hs = (ctypes.c_void_p * n)(*[l.handle.value for l in layers])
     yp = (ctypes.c_void_p * n)(*[y.data_ptr() for y in ys])
     _check(load_library().fp8_scaled_linear_multi(hs, n, M, a.data_ptr(), qa_scratch.data_ptr(),

@@ -76,3 +76,28 @@ def test_linear_create_and_forward_errors():
 def test_per_tensor_empty_errors():
     L = fp8.load_library()
     assert L.fp8_quantize_weight_per_tensor(None, 0, 0, None, 0, None) == EMPTY
+
+
+def test_binding_rejects_wrong_outputs_and_scratch():
+    """The binding checks caller-supplied outputs and scratch (dtype, shape,
+    device) before the library writes through their pointers."""
+    a = torch.zeros((8, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        fp8.quantize_rowwise(a, q=torch.empty((8, 32), dtype=torch.uint8, device="cuda"))
+    with pytest.raises(ValueError):
+        fp8.quantize_rowwise(a, scale=torch.empty((4,), dtype=torch.float32, device="cuda"))
+    layer = fp8.FP8Linear.from_weight(torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        layer.forward(a, y=torch.empty((8, 16), dtype=torch.float32, device="cuda"))
+    with pytest.raises(ValueError):
+        layer.forward(a, qa_scratch=torch.empty((4, 64), dtype=torch.uint8, device="cuda"))
+    with pytest.raises(ValueError):
+        layer.forward_weight_only(a, y=torch.empty((8, 8), dtype=torch.bfloat16, device="cuda"))
+    other = fp8.FP8Linear.from_weight(torch.zeros((16, 128), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        fp8.scaled_linear_multi([layer, other], a)  # K differs
+    with pytest.raises(ValueError):
+        fp8.scaled_linear_multi([layer], a, ys=[])
+    y = layer.forward(a)  # the defaults still work
+    torch.cuda.synchronize()
+    assert y.shape == (8, 16)
