@@ -5,6 +5,7 @@ inputs, for profiling it on its own (for example under Nsight Compute):
 
 Cases (inputs from ``synth``, the same as the benchmark's):
     quantize_ffn_up, quantize_ffn_down   rowwise E4M3 quantiser on the FFN activations
+    quantize_hidden                      rowwise E4M3 quantiser on hidden_states [32760, 2048]
     gelu_quantize_ffn_down               GELU -> E4M3 producer on a [4096, 8192] activation
     gemm_ffn_up, gemm_ffn_down           FP8 GEMM + epilogue from pre-quantised activations
     weight_only_ffn_up, ..._ffn_down     FP8 weight-only GEMM (bf16 activation)
@@ -23,7 +24,7 @@ import synth
 
 from . import E4M3FN, E5M2, FP8Linear, act_quantize_rowwise, device_error, quantize_per_tensor, quantize_rowwise
 
-CASES = ("quantize_ffn_up", "quantize_ffn_down", "gelu_quantize_ffn_down", "gemm_ffn_up", "gemm_ffn_down",
+CASES = ("quantize_ffn_up", "quantize_ffn_down", "quantize_hidden", "gelu_quantize_ffn_down", "gemm_ffn_up", "gemm_ffn_down",
          "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down", "state_dict_e4m3fn",
          "state_dict_e5m2")
 
@@ -45,8 +46,11 @@ def run(case: str, iters: int) -> None:
         if device_error() != 0:
             raise SystemExit(f"{case}: device error word set")
         return
-    workload = synth.ffn_up() if case.endswith("ffn_up") else synth.ffn_down()
-    a = _dev(workload["A"], dev)
+    if case == "quantize_hidden":
+        a = _dev(synth.attention()["hidden"], dev)
+    else:
+        workload = synth.ffn_up() if case.endswith("ffn_up") else synth.ffn_down()
+        a = _dev(workload["A"], dev)
     M, K = a.shape
     if case.startswith("quantize"):
         q = torch.empty((M, K), dtype=torch.uint8, device=dev)
