@@ -563,6 +563,39 @@ def time_region(torch, fn, iters, dev, warm=3):
     return a.elapsed_time(b) / iters
 
 
+def scaled_mm_context(torch, layer, qs, ys, M, N, K, dev):
+    """torch._scaled_mm on the layer's E4M3 codes ("rowwise": the per-token
+    and per-channel scales of the method; "tensorwise": unit scales, a
+    cheaper epilogue than the method needs), timed eagerly over 50 calls
+    (each call is longer than the host's launch cost). Records the error
+    instead of a time where this torch build refuses a scaling mode; the
+    row-scaled result is also compared with the layer's own output."""
+    res = {}
+    fa = [q.view(torch.float8_e4m3fn) for q, _ in qs]
+    fw = layer.qw.view(torch.float8_e4m3fn).t()  # [K, N], column-major
+    modes = {"rowwise": ([s.view(M, 1) for _, s in qs], layer.sw.view(1, N)),
+             "tensorwise": ([torch.ones((), dtype=torch.float32, device=dev)] * len(qs),
+                            torch.ones((), dtype=torch.float32, device=dev))}
+    for mode, (sas, sw) in modes.items():
+        try:
+            run = lambda i: torch._scaled_mm(fa[i % len(fa)], fw, scale_a=sas[i % len(fa)], scale_b=sw,
+                                             out_dtype=torch.bfloat16)
+            run(0)  # surfaces a refused mode before timing
+            ms = time_region(torch, run, 50, dev)
+            r = {"us": ms * 1e3, "tflops": 2.0 * M * N * K / (ms * 1e-3) / 1e12}
+            if mode == "rowwise":
+                # Same quantity up to the bias and two bf16 roundings.
+                layer.forward_fp8(qs[0][0], qs[0][1], y=ys[0])
+                torch.cuda.synchronize()
+                b = layer.bias.float().view(1, N) if layer.bias is not None else 0.0
+                r["max_abs_diff_vs_fp8dit"] = (run(0).float() + b - ys[0].float()).abs().max().item()
+                r["max_abs_fp8dit"] = ys[0].float().abs().max().item()
+            res[mode] = r
+        except Exception as e:  # a scaling mode this torch build does not offer
+            res[mode] = {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:160]}"}
+    return res
+
+
 def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
     out = {}
     # Attention projections: hidden [32760, 2048] quantised once, Q / K / V in one grouped launch.
@@ -667,6 +700,11 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
         bms = time_region(torch, lambda i: torch.matmul(a16, w16.t()), 50, dev)
         btf = 2.0 * M * N * K / (bms * 1e-3) / 1e12
         out[f"bf16_torch_matmul_ffn_{name}"] = {"us": bms * 1e3, "tflops": btf}
+        # FP8 library context: the same codes through torch._scaled_mm, bf16 out,
+        # no bias; bench script only. With per-row / per-column scales torch
+        # runs its own CUTLASS sm100 kernel; with one scale per operand, cuBLASLt.
+        out[f"fp8_torch_scaled_mm_ffn_{name}"] = scaled_mm_context(torch, layer, qs, ys, M, N, K, dev)
+        del a16, w16, qs, ys
     # Stream-K against the tile-per-pair schedule where the latter's last wave
     # is nearly empty: 4864 tokens x FFN-down weight = 152 tiles on 74 pairs.
     d = synth.ffn_down()
