@@ -109,11 +109,13 @@ struct alignas(64) GemmArgs {
 };
 
 // Bytes of stream-K workspace for `units` MMA units (flags, then partials).
+// The flags are indexed by the unit that finishes a tile and by its successor
+// (unit + 1 <= units), so the flag area holds units + 1 units' worth.
 constexpr size_t kSkFlagBytesPerUnit = 2 * 8 * sizeof(uint32_t);
 constexpr size_t kSkPartialBytesPerUnit = 2 * 8 * 32 * 128 * sizeof(float);
 constexpr int64_t kSkMinKBlocks = 8;  // shorter tiles gain less from a split than it costs
 inline size_t stream_k_workspace_bytes(int units) {
-    const size_t flags = ((size_t)units * kSkFlagBytesPerUnit + 4095) & ~(size_t)4095;
+    const size_t flags = ((size_t)(units + 1) * kSkFlagBytesPerUnit + 4095) & ~(size_t)4095;
     return flags + (size_t)units * kSkPartialBytesPerUnit;
 }
 
