@@ -722,6 +722,22 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
                                       "stream_k_tflops": 2.0 * M * N * K / (sk_ms * 1e-3) / 1e12,
                                       "speedup": dp_ms / sk_ms}
     del qs, ys, layer
+    # Split-K against the plain schedule for text tokens through the FFN-down
+    # weight: [26, 8192] x [2048, 8192], 16 tiles of 128 x 128.
+    M = 26
+    layer = fp8.FP8Linear.from_weight(up(d["W"]), up(d["bias"]))
+    qs = [fp8.quantize_rowwise(up(synth.normal_bf16(f"bench/split/A{i}", (M, K), 1.0))) for i in range(3)]
+    ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    run = lambda i: layer.forward_fp8(qs[i % 3][0], qs[i % 3][1], y=ys[i % 3])
+    dp_ms = graph_region_ms(torch, run, 200, dev)
+    layer.attach_workspace()
+    plan = list(layer.plan(M))
+    sp_ms = graph_region_ms(torch, run, 200, dev)
+    layer.detach_workspace()
+    out["split_k_26x2048x8192"] = {"plain_us": dp_ms * 1e3, "split_k_us": sp_ms * 1e3, "split_plan": plan,
+                                   "speedup": dp_ms / sp_ms,
+                                   "w_gbs_split": N * K / (sp_ms * 1e-3) / 1e9}
+    del qs, ys, layer
     # State-dict conversion: 192 tensors, 1.61e9 elements, both formats.
     layout = synth.state_dict_layout()
     tensors = []

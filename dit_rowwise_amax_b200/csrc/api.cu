@@ -187,12 +187,33 @@ static int choose_cfg_fused(const fp8dit_linear_s* h, int64_t M) {
     return kCfgAQ128x128;
 }
 
+// Split-K plan for the FP8 x FP8 single-CTA plans when a workspace is
+// attached: if 128 x 128 tiles fill at most half of the SMs and K has at
+// least kSplitMinKBlocksTotal k-blocks, each tile is cut into S pieces of at
+// least kSplitMinKBlocks k-blocks (S <= kSplitMaxPieces, tiles x S <= SMs), so
+// every CTA streams a short slice of W instead of one CTA per tile streaming
+// all of K. Returns S (1: no split).
+static int split_pieces(const fp8dit_linear* hs, int32_t n, int64_t M, int cfg, int num_sms) {
+    if ((cfg != kCfg128x128 && cfg != kCfg128x256) || hs[0]->sk_ws == nullptr || M <= 0) return 1;
+    int64_t tiles = 0;
+    for (int g = 0; g < n; ++g) tiles += ((M + 127) / 128) * ((hs[g]->N + 127) / 128);
+    if (tiles <= 0 || tiles * 2 > num_sms) return 1;
+    const int64_t num_kb = (hs[0]->K + 127) / 128;
+    if (num_kb < kSplitMinKBlocksTotal) return 1;
+    int64_t S = num_sms / tiles;
+    if (S > num_kb / kSplitMinKBlocks) S = num_kb / kSplitMinKBlocks;
+    if (S > kSplitMaxPieces) S = kSplitMaxPieces;
+    return S >= 2 ? (int)S : 1;
+}
+
 // a: FP8 codes [M, K] (qa) for the FP8 x FP8 configurations, bf16 [M, K] for
 // the weight-only and quantise-in-GEMM ones; sa: per-token scales, or NULL
 // (weight-only); ra: the per-token reciprocals (quantise-in-GEMM only).
 static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, const void* a, const float* sa,
                               uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev, int cfg,
                               const float* ra = nullptr) {
+    const int split = split_pieces(hs, n, M, cfg, dev->num_sms);
+    if (split > 1) cfg = kCfg128x128;
     const int bm = gemm_block_m(cfg);
     const int bn = gemm_block_n(cfg);
     const int ke = gemm_k_elems(cfg);
@@ -226,6 +247,7 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
         GemmProblem& p = args.prob[g];
         p.sw = hs[g]->sw;
         p.bias = hs[g]->bias;
+        p.y = ys[g];
         p.N = (int32_t)hs[g]->N;
         p.tiles_n = (int32_t)((hs[g]->N + bn - 1) / bn);
         p.tile_start = tiles;
@@ -239,8 +261,26 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
     // 86% busy) run 6% slower, since
     // under the power cap the SMs left idle in a data-parallel last wave let
     // the busy ones clock higher, which recovers most of the idle time.
-    const int units = gemm_units_for(cfg, tiles, dev);
+    int units = gemm_units_for(cfg, tiles, dev);
     const int64_t num_kb = (K + ke - 1) / ke;
+    if (split > 1) {
+        // One CTA per (tile, piece); tiles * split <= SMs by construction. The
+        // arrival counters and generation words (one each per tile, tiles <=
+        // SMs / 2) sit in the flag area after the stream-K flags, the partials
+        // in the partial area (tiles * split * 64 KB <= SMs * 64 KB, within
+        // (SMs / 2) * 256 KB).
+        const int pairs = hs[0]->num_sms / 2;
+        units = tiles * split;
+        if (units > dev->num_sms || (size_t)units * kSplitPieceBytes > (size_t)pairs * kSkPartialBytesPerUnit ||
+            tiles > pairs)
+            return unsupported("split-K plan exceeds the workspace");
+        args.split_k = split;
+        args.split_arrive = static_cast<uint32_t*>(hs[0]->sk_ws) + split_flag_offset_words(pairs);
+        args.split_gen = args.split_arrive + pairs;
+        args.sk_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(hs[0]->sk_ws) +
+                                                   (stream_k_workspace_bytes(pairs) -
+                                                    (size_t)pairs * kSkPartialBytesPerUnit));
+    }
     if (n == 1 && cfg == kCfgPair256 && hs[0]->sk_ws != nullptr && tiles >= units && num_kb >= kSkMinKBlocks) {
         const int64_t waves = (tiles + units - 1) / units;
         if ((waves * units - tiles) * 4 > waves * units) {
@@ -553,8 +593,11 @@ fp8dit_status fp8_linear_plan(fp8dit_linear h, int64_t M, int32_t n_problems, in
                               int32_t* ctas) {
     t_last_error[0] = 0;
     if (!h || M < 0 || n_problems < 1 || n_problems > kMaxGroups) return invalid("plan arguments");
-    const int cfg = choose_cfg(h, M, n_problems);
-    const int64_t tiles = tiles_for(h, M, n_problems, cfg);
+    int cfg = choose_cfg(h, M, n_problems);
+    const fp8dit_linear same[kMaxGroups] = {h, h, h, h};
+    const int split = split_pieces(same, n_problems, M, cfg, h->num_sms);
+    if (split > 1) cfg = kCfg128x128;
+    const int64_t tiles = tiles_for(h, M, n_problems, cfg) * split;
     const int64_t max_units = h->num_sms / gemm_cta_group(cfg);
     if (block_m) *block_m = gemm_block_m(cfg);
     if (block_n) *block_n = gemm_block_n(cfg);

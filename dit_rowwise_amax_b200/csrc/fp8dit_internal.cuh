@@ -81,6 +81,7 @@ constexpr int kMaxGroups = 4;
 struct GemmProblem {
     const float* sw;
     const uint16_t* bias;  // may be null
+    uint16_t* y;           // bf16 [M, N], row-major (split-K stores it directly)
     int32_t N;
     int32_t tiles_n;
     int32_t tile_start;  // first global tile index of this problem
@@ -104,18 +105,45 @@ struct alignas(64) GemmArgs {
     // first, stores the fp32 partial in sk_partial and sets sk_flag to 1; u
     // waits for 1, adds the partial and clears the flag again.
     int32_t stream_k;
-    uint32_t* sk_flag;   // [units][2 CTAs][8 epilogue warps]
-    float* sk_partial;   // [units][2 CTAs][8 epilogue warps][32 rows][128 columns]
+    // Split-K (128 x 128 single-CTA tiles, few tiles): split_k > 1 pieces per
+    // tile, CTA u computing piece u % split_k of tile u / split_k over an equal
+    // share of the k-blocks. Every piece stores its fp32 partial and arrives on
+    // the tile's counter; the last arrival resets the counter and advances the
+    // tile's generation word, which the other pieces wait for; then each
+    // piece's CTA adds the split_k partials in piece order for its share of
+    // the tile's rows and writes y.
+    int32_t split_k;
+    uint32_t* split_arrive;  // split-K: arrival counter per tile (zero between launches)
+    uint32_t* split_gen;     // split-K: generation word per tile (any value)
+    uint32_t* sk_flag;   // stream-K: [units + 1][2 CTAs][8 epilogue warps] (zero between launches)
+    float* sk_partial;   // stream-K: [units][2 CTAs][8 epilogue warps][32 rows][128 columns];
+                         // split-K: [tiles][split_k][4 quarters][2 halves][16 float4][32 rows]
 };
 
-// Bytes of stream-K workspace for `units` MMA units (flags, then partials).
-// The flags are indexed by the unit that finishes a tile and by its successor
-// (unit + 1 <= units), so the flag area holds units + 1 units' worth.
+// Stream-K / split-K workspace for `units` CTA pairs: a flag area, then the
+// partials. The flag area holds the stream-K flags ((units + 1) x 16 words,
+// indexed by the unit that finishes a tile and its successor), then the
+// split-K arrival counters and generation words (units each: a split launch
+// has at most one tile per pair). Every region starts zeroed by
+// fp8_linear_set_workspace; stream-K flags and arrival counters return to
+// zero at the end of every launch, so one workspace serves any sequence of
+// stream-ordered launches of either schedule.
 constexpr size_t kSkFlagBytesPerUnit = 2 * 8 * sizeof(uint32_t);
+inline size_t sk_flag_words(int units) { return (size_t)(units + 1) * 16; }
+inline size_t split_flag_offset_words(int units) { return sk_flag_words(units); }
 constexpr size_t kSkPartialBytesPerUnit = 2 * 8 * 32 * 128 * sizeof(float);
 constexpr int64_t kSkMinKBlocks = 8;  // shorter tiles gain less from a split than it costs
+// Split-K pays where a single-CTA tile's k-loop, which at small M is bound by
+// the ring's turnover (~1.7 us per 6 k-blocks on B200), is much longer than
+// the split's fixed cost (~3.5 us: partial stores, the arrival handshake
+// across the GPU, the reduction). Measured: K = 8192 (64 k-blocks) runs 2.1x
+// faster at M <= 26 and 1.55x at M = 128; K = 2048 gains nothing.
+constexpr int kSplitMinKBlocksTotal = 48;  // split-K: k-blocks of the layer, at least
+constexpr int kSplitMinKBlocks = 6;        // split-K: k-blocks per piece (one ring), at least
+constexpr int kSplitMaxPieces = 8;         // split-K: pieces per tile, at most
+constexpr size_t kSplitPieceBytes = 128 * 128 * sizeof(float);  // one fp32 128 x 128 partial
 inline size_t stream_k_workspace_bytes(int units) {
-    const size_t flags = ((size_t)(units + 1) * kSkFlagBytesPerUnit + 4095) & ~(size_t)4095;
+    const size_t flags = ((sk_flag_words(units) + 2 * (size_t)units) * sizeof(uint32_t) + 4095) & ~(size_t)4095;
     return flags + (size_t)units * kSkPartialBytesPerUnit;
 }
 

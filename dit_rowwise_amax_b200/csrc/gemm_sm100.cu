@@ -41,7 +41,9 @@
 // Schedules: data-parallel (tile t on MMA unit t mod units) or, with a
 // workspace, stream-K (each unit an equal share of all k-blocks; a tile split
 // between two units is finished by one of them after the other has published
-// its fp32 partial), see SegSched.
+// its fp32 partial) or split-K for few tiles and a long K (one CTA per (tile,
+// piece of K); once every piece has stored its fp32 partial, each adds the
+// pieces in order for its share of the rows), see SegSched.
 //
 // Every mbarrier wait is bounded (mbar_wait_bounded): on expiry the CTA
 // raises the device error word and its own and its peer's abort flags, lets
@@ -87,6 +89,8 @@ struct Cfg {
     static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
     static constexpr int EPI_WARPS = CONV ? 4 : 8;   // one or two per TMEM lane quarter
+    // Split-K is compiled only into the FP8 128 x 128 single-CTA kernel.
+    static constexpr bool SPLIT_OK = CG == 1 && BN == 128 && OPS == kOpsFp8;
     static constexpr int CONV_WARPS = CONV ? STAGES : 0;  // converter warps, one per ring stage
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
     static constexpr int BOX = 32;                   // epilogue store box: 32 rows x 32 columns
@@ -98,7 +102,7 @@ struct Cfg {
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_SMEM + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
     static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-    static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
+    static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 20 <= BAR_BYTES, "barrier area");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(!W8 || (B_BYTES == 2 * RAW_BYTES && B_ROWS == 128), "in-place decode layout");
     static_assert(!AQ || ROWS == 128, "in-place quantise layout");
@@ -122,20 +126,27 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
 // unit's equal share [pos, end) of the num_tiles x num_kb k-blocks, cut at
 // tile boundaries. With num_tiles >= units a share spans at least one tile,
 // so a tile has at most two segments: a head [0, a) that ends its unit's
-// share and a tail [a, num_kb) that starts the next unit's share.
+// share and a tail [a, num_kb) that starts the next unit's share. Split-K:
+// piece p of tile t (work item t * split + p, items dealt round-robin) covers
+// k-blocks [p * num_kb / split, (p + 1) * num_kb / split).
 struct Segment {
-    int t, k0, k1;
+    int t, k0, k1, piece;
 };
 struct SegSched {
     int64_t pos, end;
-    int step, num_kb;
+    int step, num_kb, split;
     bool sk;
 };
-__device__ __forceinline__ SegSched seg_begin(const GemmArgs& a, int unit, int units) {
+__device__ __forceinline__ SegSched seg_begin(const GemmArgs& a, int unit, int units, bool split_ok) {
     SegSched s;
     s.sk = a.stream_k != 0;
     s.num_kb = a.num_kb;
-    if (s.sk) {
+    s.split = split_ok && a.split_k > 1 ? a.split_k : 1;
+    if (s.split > 1) {
+        s.pos = unit;
+        s.end = (int64_t)a.num_tiles * s.split;
+        s.step = units;
+    } else if (s.sk) {
         const int64_t total = (int64_t)a.num_tiles * a.num_kb;
         s.pos = total * unit / units;
         s.end = total * (unit + 1) / units;
@@ -149,7 +160,14 @@ __device__ __forceinline__ SegSched seg_begin(const GemmArgs& a, int unit, int u
 }
 __device__ __forceinline__ bool seg_next(SegSched& s, Segment& g) {
     if (s.pos >= s.end) return false;
-    if (s.sk) {
+    g.piece = 0;
+    if (s.split > 1) {
+        g.t = (int)(s.pos / s.split);
+        g.piece = (int)(s.pos % s.split);
+        g.k0 = (int)((int64_t)g.piece * s.num_kb / s.split);
+        g.k1 = (int)((int64_t)(g.piece + 1) * s.num_kb / s.split);
+        s.pos += s.step;
+    } else if (s.sk) {
         g.t = (int)(s.pos / s.num_kb);
         g.k0 = (int)(s.pos % s.num_kb);
         const int64_t tile_end = (int64_t)(g.t + 1) * s.num_kb;
@@ -169,6 +187,11 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu_u32(const uint32_t* p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+__device__ __forceinline__ uint32_t atom_acq_rel_gpu_add_u32(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 __device__ __forceinline__ void st_release_gpu_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -200,6 +223,9 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     uint64_t* drain = tempty + C::ACC;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile uint32_t* split_ticket = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);  // split-K
+    volatile uint32_t* split_fail = reinterpret_cast<volatile uint32_t*>(tmem_slot + 3);    // split-K
+    volatile uint32_t* split_gen = reinterpret_cast<volatile uint32_t*>(tmem_slot + 4);     // split-K
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -225,6 +251,9 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
+        *split_ticket = 0u;
+        *split_fail = 0u;
+        *split_gen = 0u;
         fence_mbarrier_init();
         tma_prefetch_desc(&args.tmA);
         for (int g = 0; g < args.G; ++g) {
@@ -257,7 +286,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
         if (lane == 0) {
             uint32_t stage = 0, phase = 0;
             int64_t armed = 0;
-            SegSched ss = seg_begin(args, unit, units);
+            SegSched ss = seg_begin(args, unit, units, C::SPLIT_OK);
             Segment sg;
             while (!aborted && seg_next(ss, sg)) {
                 const TileCoord tc = tile_coord(args, sg.t);
@@ -309,7 +338,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
         if (lane == 0 && leader) {
             constexpr uint32_t idesc = W8 ? umma_idesc_bf16_f32(C::BM, BN) : umma_idesc_e4m3_f32(C::BM, BN);
             uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-            SegSched ss = seg_begin(args, unit, units);
+            SegSched ss = seg_begin(args, unit, units, C::SPLIT_OK);
             Segment sg;
             while (!aborted && seg_next(ss, sg)) {
                 if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, args.err)) {
@@ -426,10 +455,69 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             }
         };
 
+        // Split-K: once all pieces of tile t are stored, this CTA (piece p of
+        // S) adds, for rows [p R / S, (p + 1) R / S) of the tile's R valid
+        // rows, the S partials in piece order, applies the epilogue and stores
+        // bf16 to y. Thread i takes items i, i + 256, ...: item = (row, column
+        // float4 f), f fastest, so a warp's y stores are contiguous.
+        auto split_reduce = [&](int t, int p) {
+            const TileCoord tc = tile_coord(args, t);
+            const GemmProblem& P = args.prob[tc.g];
+            const int r0 = tc.tm * C::BM;
+            const int rows = args.M - r0 < C::BM ? args.M - r0 : C::BM;
+            const int c0 = tc.tn * BN;
+            const int cols = P.N - c0 < BN ? P.N - c0 : BN;
+            const int S = args.split_k;
+            const int ra = (int)((int64_t)p * rows / S);
+            const int rb = (int)((int64_t)(p + 1) * rows / S);
+            constexpr int F4 = BN / 4;                        // float4 columns per row
+            constexpr size_t PIECE4 = (size_t)C::ROWS * BN / 4;  // float4 per piece
+            const float4* base = reinterpret_cast<const float4*>(args.sk_partial) + (size_t)t * S * PIECE4;
+            const int n_items = (rb - ra) * F4;
+            for (int i = ew * 32 + lane; i < n_items; i += 32 * C::EPI_WARPS) {
+                const int r = ra + i / F4;
+                const int f = i % F4;
+                if (4 * f >= cols) continue;
+                // Partial layout of a piece: [quarter q][column half h][chunk float4 cv][row lane].
+                const int off = ((((r >> 5) * 2 + f / (C::EPI_COLS / 4)) * (C::EPI_COLS / 4) + f % (C::EPI_COLS / 4)) << 5) + (r & 31);
+                // Pieces in groups of four loads in flight, added in piece order.
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int g = 0; g < kSplitMaxPieces; g += 4) {
+                    if (g >= S) break;
+                    float4 x[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (g + k < S) x[k] = __ldcg(base + (size_t)(g + k) * PIECE4 + off);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (g + k < S) {
+                            v.x += x[k].x;
+                            v.y += x[k].y;
+                            v.z += x[k].z;
+                            v.w += x[k].w;
+                        }
+                    }
+                }
+                const float sa = args.sa != nullptr ? __ldg(args.sa + r0 + r) : 1.0f;
+                const int n = c0 + 4 * f;
+                const float4 w4 = __ldg(reinterpret_cast<const float4*>(P.sw + n));
+                uint2 b2 = make_uint2(0u, 0u);
+                if (P.bias != nullptr) b2 = __ldg(reinterpret_cast<const uint2*>(P.bias + n));
+                const float o0 = fmaf(v.x * sa, w4.x, __uint_as_float(b2.x << 16));
+                const float o1 = fmaf(v.y * sa, w4.y, __uint_as_float(b2.x & 0xffff0000u));
+                const float o2 = fmaf(v.z * sa, w4.z, __uint_as_float(b2.y << 16));
+                const float o3 = fmaf(v.w * sa, w4.w, __uint_as_float(b2.y & 0xffff0000u));
+                *reinterpret_cast<uint2*>(P.y + (size_t)(r0 + r) * P.N + n) =
+                    make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+            }
+        };
+
         uint32_t acc = 0, acc_phase = 0;
         uint32_t stores = 0;
+        const bool split = C::SPLIT_OK && args.split_k > 1;
         Pre pre;
-        SegSched ss = seg_begin(args, unit, units);
+        SegSched ss = seg_begin(args, unit, units, C::SPLIT_OK);
         SegSched look = ss;  // one segment ahead, for the operand prefetch
         Segment sg, nx;
         bool has_next = seg_next(look, nx);
@@ -448,8 +536,11 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             // partial (32 rows x EPI_COLS fp32) is stored lane-fastest: float4 v
             // of row `lane` in column chunk c sits at [(c * 8 + v) * 32 + lane],
             // so every warp access moves 512 contiguous bytes.
-            const bool tail = sg.k0 > 0;
-            const bool head = sg.k0 == 0 && sg.k1 < args.num_kb;
+            // Split-K: the tile's generation before this piece arrives (read
+            // while the accumulator is still being built).
+            if (split && ew == 0 && lane == 0) *split_gen = ld_acquire_gpu_u32(args.split_gen + sg.t);
+            const bool tail = !split && sg.k0 > 0;
+            const bool head = !split && sg.k0 == 0 && sg.k1 < args.num_kb;
             const size_t part_elems = 32 * C::EPI_COLS;
             float4* my_part = nullptr;
             const float4* their_part = nullptr;
@@ -490,20 +581,38 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             // Every lane waits; the warp then agrees (and reconverges) before
             // the warp-collective TMEM loads.
             const bool ready = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, args.err);
+            bool failed = false;
             if (!__all_sync(0xffffffffu, ready)) {
                 if (lane == 0) abort_peer();
-                break;
+                if (!split) break;
+                failed = true;  // split-K: still meet the CTA's epilogue barriers below
             }
             tc_fence_after();
             const int n_tile = args.prob[tc.g].N;
             const uint32_t t_addr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + col0;
 #pragma unroll 1
-            for (int c = 0; c < C::EPI_COLS / 32; ++c) {
+            for (int c = 0; c < (failed ? 0 : C::EPI_COLS / 32); ++c) {
                 const int n0 = tc.tn * BN + col0 + c * 32;
                 if (n0 >= n_tile) break;  // warp-uniform
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_addr + c * 32, r);
                 tmem_wait_ld();
+                if (split) {
+                    // This piece's raw fp32 partial, [q][half][chunk float4][lane]:
+                    // every warp store moves 512 contiguous bytes. Warps whose
+                    // rows all lie past M store nothing (nothing reads them).
+                    if (row0 < args.M) {
+                        float4* dst = reinterpret_cast<float4*>(args.sk_partial) +
+                                      (size_t)((int64_t)sg.t * args.split_k + sg.piece) * (C::ROWS * BN / 4) +
+                                      ((((size_t)q * 2 + (ew >> 2)) * (C::EPI_COLS / 4) + c * 8) << 5) + lane;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            __stcg(dst + v * 32,
+                                   make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+                    }
+                    continue;
+                }
                 if (tail) {
                     // Raw fp32 accumulator of this piece: row `lane`, columns c*32..+31.
 #pragma unroll
@@ -583,6 +692,47 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 acc = 0;
                 acc_phase ^= 1u;
             }
+            if (split) {
+                // After all of this CTA's partial stores, thread 0 arrives on
+                // the tile's counter (acquire-release). The arrival that
+                // completes the count resets the counter and bumps the tile's
+                // generation word (release); every other piece waits, bounded,
+                // for the generation to move past the value it read before
+                // arriving. Then each piece reduces its share of the rows. The
+                // grid has one CTA per (tile, piece), at most one per SM, and
+                // each CTA allows the dependent launch only once it runs, so
+                // every piece is resident before any wait can matter. Every
+                // epilogue warp reaches every barrier on every path.
+                uint32_t* arrive = args.split_arrive + sg.t;
+                uint32_t* gen = args.split_gen + sg.t;
+                if (failed && lane == 0) *split_fail = 1u;
+                named_barrier_sync(1, 32 * C::EPI_WARPS);
+                if (ew == 0 && lane == 0) {
+                    bool ok = *split_fail == 0u;
+                    if (ok) {
+                        const uint32_t gen0 = *split_gen;
+                        if (atom_acq_rel_gpu_add_u32(arrive, 1u) == (uint32_t)args.split_k - 1u) {
+                            *arrive = 0u;
+                            st_release_gpu_u32(gen, gen0 + 1u);
+                        } else {
+                            const unsigned long long t0 = globaltimer_ns();
+                            while (ld_acquire_gpu_u32(gen) == gen0) {
+                                if (globaltimer_ns() - t0 > args.err.limit_ns) {
+                                    atomicOr(args.err.word, kDevErrTimeout);
+                                    ok = false;
+                                    break;
+                                }
+                                __nanosleep(32);
+                            }
+                        }
+                    }
+                    *split_ticket = ok ? 1u : 0u;
+                }
+                named_barrier_sync(1, 32 * C::EPI_WARPS);
+                if (*split_ticket == 1u) {
+                    if constexpr (C::SPLIT_OK) split_reduce(sg.t, sg.piece);
+                }
+            }
         }
         if (lane == 0) bulk_wait_group<0>();  // all output stores complete
         __syncwarp();
@@ -605,7 +755,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             const int own = warp - (2 + C::EPI_WARPS);     // the stage this warp decodes
             uint32_t stage = 0, phase = 0;
             bool stop = false;
-            SegSched ss = seg_begin(args, unit, units);
+            SegSched ss = seg_begin(args, unit, units, C::SPLIT_OK);
             Segment sg;
             while (!stop && seg_next(ss, sg)) {
                 for (int kb = sg.k0; kb < sg.k1; ++kb) {
@@ -680,7 +830,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             const int own = warp - (2 + C::EPI_WARPS);
             uint32_t stage = 0, phase = 0;
             bool stop = false;
-            SegSched ss = seg_begin(args, unit, units);
+            SegSched ss = seg_begin(args, unit, units, C::SPLIT_OK);
             Segment sg;
             while (!stop && seg_next(ss, sg)) {
                 const TileCoord tc = tile_coord(args, sg.t);

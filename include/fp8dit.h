@@ -180,14 +180,22 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  * an equal share of the layer's k-blocks; a tile split between two pairs is
  * finished by one of them after the other has stored its fp32 partial in this
  * workspace. Results stay deterministic (the two parts are added once, in
- * fp32) but differ in rounding from the plain schedule. Without a workspace,
- * or for other shapes (the FFN shapes among them), the plain schedule is used.
+ * fp32) but differ in rounding from the plain schedule.
+ * The same workspace enables split-K for few tiles and a long K: when the
+ * 128 x 128 tiles of a small-M call fill at most half of the SMs and K has at
+ * least 48 k-blocks (K >= 6144; e.g. text tokens through an FFN-down weight),
+ * each tile is cut into up to 8 pieces of at least 6 k-blocks on separate
+ * CTAs; the pieces' fp32 partials are added in piece order (deterministic,
+ * rounding differs from the plain schedule). fp8_scaled_linear_multi uses the
+ * workspace of its first layer. Without a workspace, or for other shapes (the
+ * FFN shapes among them), the plain schedule is used.
  *   fp8_linear_workspace_size: bytes needed on the layer's device (~19 MB on
  *     148 SMs), the same for every M.
  *   fp8_linear_set_workspace: attach caller-owned DEVICE memory (256-byte
  *     aligned, at least that size) or detach with NULL, while no call that
  *     uses the layer is in flight. Attaching clears the workspace's flags
- *     (synchronously); every launch leaves them cleared, so
+ *     (synchronously); every launch leaves them cleared (split-K's
+ *     generation words excepted, which may hold any value), so
  *     stream-ordered launches and replays of a captured CUDA graph need no
  *     host reset. After a call whose device error word reports
  *     FP8DIT_ERR_TIMEOUT, attach the workspace again before reusing it. The
