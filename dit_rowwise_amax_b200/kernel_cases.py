@@ -10,6 +10,8 @@ Cases (inputs from ``synth``, the same as the benchmark's):
     gemm_ffn_up, gemm_ffn_down           FP8 GEMM + epilogue from pre-quantised activations
     weight_only_ffn_up, ..._ffn_down     FP8 weight-only GEMM (bf16 activation)
     fused_ffn_up, fused_ffn_down         quantise-in-GEMM variant (row-scale pre-pass + GEMM)
+    gemm_text_ffn_down                   FP8 GEMM, 26 tokens x FFN-down weight, plain schedule
+    split_k_text_ffn_down                the same with a workspace attached (split-K schedule)
     state_dict_e4m3fn, state_dict_e5m2   per-tensor conversion of the 192-tensor DiT weight set
 Layer creation runs the per-channel weight quantiser first; every case then
 launches only its own kernels. Exits non-zero if the device reports an error.
@@ -25,8 +27,9 @@ import synth
 from . import E4M3FN, E5M2, FP8Linear, act_quantize_rowwise, device_error, quantize_per_tensor, quantize_rowwise
 
 CASES = ("quantize_ffn_up", "quantize_ffn_down", "quantize_hidden", "gelu_quantize_ffn_down", "gemm_ffn_up", "gemm_ffn_down",
-         "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down", "state_dict_e4m3fn",
-         "state_dict_e5m2")
+         "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down", "gemm_text_ffn_down",
+         "split_k_text_ffn_down", "state_dict_e4m3fn", "state_dict_e5m2")
+TEXT_TOKENS = 26  # encoder_hidden_states length
 
 
 def _dev(a: np.ndarray, dev) -> torch.Tensor:
@@ -50,7 +53,8 @@ def run(case: str, iters: int) -> None:
         a = _dev(synth.attention()["hidden"], dev)
     else:
         workload = synth.ffn_up() if case.endswith("ffn_up") else synth.ffn_down()
-        a = _dev(workload["A"], dev)
+        rows = workload["A"][:TEXT_TOKENS] if "_text_" in case else workload["A"]
+        a = _dev(rows, dev)
     M, K = a.shape
     if case.startswith("quantize"):
         q = torch.empty((M, K), dtype=torch.uint8, device=dev)
@@ -65,7 +69,9 @@ def run(case: str, iters: int) -> None:
     else:
         layer = FP8Linear.from_weight(_dev(workload["W"], dev), _dev(workload["bias"], dev))
         y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=dev)
-        if case.startswith("gemm"):
+        if case.startswith("split_k"):
+            layer.attach_workspace()
+        if case.startswith("gemm") or case.startswith("split_k"):
             qa, sa = quantize_rowwise(a)
             for _ in range(iters):
                 layer.forward_fp8(qa, sa, y=y)
