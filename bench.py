@@ -611,7 +611,9 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
     qb = 3 * M * 2048 + 4 * M
     out["quantizer_hidden"] = {"us": qms * 1e3, "gbs": qb / (qms * 1e-3) / 1e9,
                                "frac_of_hbm": qb / (qms * 1e-3) / 1e9 / hbm_peak}
-    for name in ("hidden", "encoder"):
+    # encoder_hidden_states first: its ~10 us launches are latency-bound and
+    # read slower in the power state the hidden_states projections leave.
+    for name in ("encoder", "hidden"):
         A = [up(att[name]) for _ in range(2)]
         M = att[name].shape[0]
         qa = torch.empty((M, 2048), dtype=torch.uint8, device=dev)

@@ -164,11 +164,16 @@ static int64_t tiles_for(const fp8dit_linear_s* h, int64_t M, int n_problems, in
 //  - 256 x 256 tiles on CTA pairs when M fills a pair tile and the tiles keep
 //    at least half of the pairs busy;
 //  - else 128 x 256 tiles on single CTAs when they keep half the SMs busy;
-//  - else 128 x 128 tiles (small M: more CTAs, shorter latency).
+//  - else 128 x 64 tiles when they fit in one wave (small M: the most CTAs,
+//    the deepest ring, the shortest epilogue);
+//  - else 128 x 128 tiles.
 static int choose_cfg(const fp8dit_linear_s* h, int64_t M, int n_problems) {
     const int pairs = h->num_sms / 2;
     if (M >= 256 && tiles_for(h, M, n_problems, kCfgPair256) * 2 >= pairs) return kCfgPair256;
     if (tiles_for(h, M, n_problems, kCfg128x256) * 2 >= h->num_sms) return kCfg128x256;
+    // Few tiles: 128 x 64 tiles while they fit in one wave (twice the CTAs,
+    // an 8-deep ring and half the epilogue per CTA of a 128 x 128 tile).
+    if (tiles_for(h, M, n_problems, kCfg128x64) <= h->num_sms) return kCfg128x64;
     return kCfg128x128;
 }
 
@@ -194,7 +199,8 @@ static int choose_cfg_fused(const fp8dit_linear_s* h, int64_t M) {
 // every CTA streams a short slice of W instead of one CTA per tile streaming
 // all of K. Returns S (1: no split).
 static int split_pieces(const fp8dit_linear* hs, int32_t n, int64_t M, int cfg, int num_sms) {
-    if ((cfg != kCfg128x128 && cfg != kCfg128x256) || hs[0]->sk_ws == nullptr || M <= 0) return 1;
+    if ((cfg != kCfg128x128 && cfg != kCfg128x256 && cfg != kCfg128x64) || hs[0]->sk_ws == nullptr || M <= 0)
+        return 1;
     int64_t tiles = 0;
     for (int g = 0; g < n; ++g) tiles += ((M + 127) / 128) * ((hs[g]->N + 127) / 128);
     if (tiles <= 0 || tiles * 2 > num_sms) return 1;
@@ -204,6 +210,13 @@ static int split_pieces(const fp8dit_linear* hs, int32_t n, int64_t M, int cfg, 
     if (S > num_kb / kSplitMinKBlocks) S = num_kb / kSplitMinKBlocks;
     if (S > kSplitMaxPieces) S = kSplitMaxPieces;
     return S >= 2 ? (int)S : 1;
+}
+
+// Rows of A per TMA load for the FP8 x FP8 plans. With one row tile on a
+// single CTA only M rows (rounded up to 8) are loaded: zero-filling the rest
+// of a 128-row box slowed 96 CTAs at M = 26 from 7.7 to 10 us per launch.
+static int a_box_rows_for(int cfg, int64_t M) {
+    return (gemm_cta_group(cfg) == 1 && M < 128) ? (int)((M + 7) / 8 * 8) : 128;
 }
 
 // a: FP8 codes [M, K] (qa) for the FP8 x FP8 configurations, bf16 [M, K] for
@@ -230,8 +243,9 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
         : gemm_quantizes_a(cfg)
             ? encode_tma_2d(&args.tmA, 2, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, (uint32_t)ke, 128,
                             CU_TENSOR_MAP_SWIZZLE_NONE)
-            : encode_tma_2d(&args.tmA, 1, a, (uint64_t)K, (uint64_t)M, (uint64_t)K, (uint32_t)ke, 128,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
+            : encode_tma_2d(&args.tmA, 1, a, (uint64_t)K, (uint64_t)M, (uint64_t)K, (uint32_t)ke,
+                            (uint32_t)a_box_rows_for(cfg, M), CU_TENSOR_MAP_SWIZZLE_128B);
+    args.a_box_rows = a_box_rows_for(cfg, M);
     if (st != FP8DIT_OK) return st;
     const int64_t tiles_m64 = (M + bm - 1) / bm;
     int64_t tiles64 = 0;

@@ -113,6 +113,11 @@ struct alignas(64) GemmArgs {
     // piece's CTA adds the split_k partials in piece order for its share of
     // the tile's rows and writes y.
     int32_t split_k;
+    // Rows of A one TMA load brings per stage in the single-CTA FP8 plans:
+    // M rounded up to 8 when M < 128 (one row tile), else 128. The MMA still
+    // reads 128 rows; rows past the box hold stale data and only feed
+    // accumulator rows past M, which are never stored.
+    int32_t a_box_rows;
     uint32_t* split_arrive;  // split-K: arrival counter per tile (zero between launches)
     uint32_t* split_gen;     // split-K: generation word per tile (any value)
     uint32_t* sk_flag;   // stream-K: [units + 1][2 CTAs][8 epilogue warps] (zero between launches)
@@ -156,7 +161,8 @@ enum GemmConfig : int32_t {
     kCfgW8128x128 = 4,  // bf16 x FP8 weight (weight-only): 128 x 128 tile on one CTA
     kCfgAQPair256 = 5,  // bf16 A quantised in the GEMM x FP8 weight: 256 x 256 tile on a 2-CTA pair
     kCfgAQ128x128 = 6,  // bf16 A quantised in the GEMM x FP8 weight: 128 x 128 tile on one CTA
-    kNumCfgs = 7,
+    kCfg128x64 = 7,     // FP8 x FP8: 128 x 64 tile on one CTA (few rows: deeper ring, more CTAs)
+    kNumCfgs = 8,
 };
 int gemm_block_m(int cfg);
 int gemm_block_n(int cfg);

@@ -85,7 +85,7 @@ struct Cfg {
     static constexpr int RAW_BYTES = W8 ? B_ROWS * 64 : 0;
     static constexpr int TX_BYTES = A_STAGE + (W8 ? RAW_BYTES : B_BYTES);  // TMA bytes per CTA per stage
     static constexpr int STAGE_SMEM = A_STAGE + B_BYTES;
-    static constexpr int STAGES = W8 ? 6 : AQ ? 4 : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : 6));
+    static constexpr int STAGES = W8 ? 6 : AQ ? 4 : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : BN == 64 ? 8 : 6));
     static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
     static constexpr int EPI_WARPS = CONV ? 4 : 8;   // one or two per TMEM lane quarter
@@ -101,7 +101,7 @@ struct Cfg {
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_SMEM + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
-    static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+    static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
     static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 20 <= BAR_BYTES, "barrier area");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(!W8 || (B_BYTES == 2 * RAW_BYTES && B_ROWS == 128), "in-place decode layout");
@@ -312,7 +312,8 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                         tma_load_2d_pair(sA + stage * C::A_STAGE, &args.tmA, bar, kb * C::KE, a_row);
                         tma_load_2d_pair(sB + stage * C::B_BYTES, &args.tmB[tc.g], bar, kb * C::KE, b_row);
                     } else {
-                        mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                        // Single CTA: A brings args.a_box_rows rows (M < 128) or 128.
+                        mbar_arrive_expect_tx(&full[stage], args.a_box_rows * C::ROW_BYTES + C::B_BYTES);
                         tma_load_2d(sA + stage * C::A_STAGE, &args.tmA, &full[stage], kb * C::KE, a_row);
                         tma_load_2d(sB + stage * C::B_BYTES, &args.tmB[tc.g], &full[stage], kb * C::KE, b_row);
                     }
@@ -925,8 +926,10 @@ int gemm_cta_group(int cfg) {
     return (cfg == kCfgPair256 || cfg == kCfgW8Pair256 || cfg == kCfgAQPair256) ? 2 : 1;
 }
 int gemm_block_m(int cfg) { return 128 * gemm_cta_group(cfg); }
-int gemm_block_n(int cfg) { return (cfg == kCfg128x128 || cfg == kCfgW8128x128 || cfg == kCfgAQ128x128) ? 128 : 256; }
-int gemm_b_box_rows(int cfg) { return cfg == kCfg128x256 ? 256 : 128; }
+int gemm_block_n(int cfg) {
+    return cfg == kCfg128x64 ? 64 : (cfg == kCfg128x128 || cfg == kCfgW8128x128 || cfg == kCfgAQ128x128) ? 128 : 256;
+}
+int gemm_b_box_rows(int cfg) { return cfg == kCfg128x256 ? 256 : cfg == kCfg128x64 ? 64 : 128; }
 bool gemm_weight_only(int cfg) { return cfg == kCfgW8Pair256 || cfg == kCfgW8128x128; }
 bool gemm_quantizes_a(int cfg) { return cfg == kCfgAQPair256 || cfg == kCfgAQ128x128; }
 int gemm_k_elems(int cfg) { return gemm_weight_only(cfg) ? 64 : 128; }
@@ -953,6 +956,8 @@ cudaError_t launch_gemm(int cfg, const GemmArgs& args, int units, cudaStream_t s
             return launch_cfg<2, 256, kOpsAQ>(args, units, stream);
         case kCfgAQ128x128:
             return launch_cfg<1, 128, kOpsAQ>(args, units, stream);
+        case kCfg128x64:
+            return launch_cfg<1, 64, kOpsFp8>(args, units, stream);
         default:
             return cudaErrorInvalidValue;
     }

@@ -187,4 +187,4 @@ def test_plan_is_reported():
     d = synth.ffn_up()
     layer, _, _ = make_layer(d["W"][:256], d["bias"][:256])
     bm, bn, ctas = layer.plan(4096)
-    assert bm == 128 and bn in (128, 256) and ctas >= 1
+    assert bm == 128 and bn in (64, 128, 256) and ctas >= 1
