@@ -134,9 +134,10 @@ def test_multi_equals_single_calls_attention_full_size():
             check_full(y, qao, sao, qw, sw, b)  # all 32760 x 2048 outputs of each projection
 
 
-def test_multi_two_and_four_layers_with_different_n():
+@pytest.mark.parametrize("M", [26, 333])  # one row tile (A loaded as 32 rows) / three row tiles
+def test_multi_two_and_four_layers_with_different_n(M):
     K = 512
-    A = synth.normal_bf16("gpu/multi/A", (333, K), 1.0)
+    A = synth.normal_bf16("gpu/multi/A" if M == 333 else f"gpu/multi/A{M}", (M, K), 1.0)
     layers, refs = [], []
     for i, N in enumerate((256, 520, 136, 1024)):
         W = synth.normal_bf16(f"gpu/multi/W{i}", (N, K), 0.02)
@@ -147,10 +148,15 @@ def test_multi_two_and_four_layers_with_different_n():
     x = to_device_bf16(A)
     qao, sao = oracle.quantize_rows(A, oracle.E4M3FN)
     for n in (2, 4):
+        assert layers[0].plan(M, n)[:2] == (128, 64)  # the tiles of all n layers fit one wave
         ys = fp8.scaled_linear_multi(layers[:n], x)
         torch.cuda.synchronize()
         for y, (qw, sw, b) in zip(ys, refs[:n]):
             check_full(y, qao, sao, qw, sw, b)
+        singles = [layer.forward(x) for layer in layers[:n]]
+        torch.cuda.synchronize()
+        for y, s1 in zip(ys, singles):
+            assert torch.equal(y.view(torch.int16), s1.view(torch.int16))
 
 
 def test_output_canaries():
