@@ -731,15 +731,21 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
     qs = [fp8.quantize_rowwise(up(synth.normal_bf16(f"bench/split/A{i}", (M, K), 1.0))) for i in range(3)]
     ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(3)]
     run = lambda i: layer.forward_fp8(qs[i % 3][0], qs[i % 3][1], y=ys[i % 3])
+    a16s = [up(synth.normal_bf16(f"bench/split/A16_{i}", (M, K), 1.0)) for i in range(3)]
+    run_wo = lambda i: layer.forward_weight_only(a16s[i % 3], y=ys[i % 3])
     dp_ms = graph_region_ms(torch, run, 200, dev)
+    wo_ms = graph_region_ms(torch, run_wo, 200, dev)
     layer.attach_workspace()
     plan = list(layer.plan(M))
     sp_ms = graph_region_ms(torch, run, 200, dev)
+    wos_ms = graph_region_ms(torch, run_wo, 200, dev)
     layer.detach_workspace()
     out["split_k_26x2048x8192"] = {"plain_us": dp_ms * 1e3, "split_k_us": sp_ms * 1e3, "split_plan": plan,
                                    "speedup": dp_ms / sp_ms,
-                                   "w_gbs_split": N * K / (sp_ms * 1e-3) / 1e9}
-    del qs, ys, layer
+                                   "w_gbs_split": N * K / (sp_ms * 1e-3) / 1e9,
+                                   "weight_only_plain_us": wo_ms * 1e3, "weight_only_split_k_us": wos_ms * 1e3,
+                                   "weight_only_speedup": wo_ms / wos_ms}
+    del qs, ys, layer, a16s
     # State-dict conversion: 192 tensors, 1.61e9 elements, both formats.
     layout = synth.state_dict_layout()
     tensors = []

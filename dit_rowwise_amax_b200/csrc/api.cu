@@ -192,20 +192,27 @@ static int choose_cfg_fused(const fp8dit_linear_s* h, int64_t M) {
     return kCfgAQ128x128;
 }
 
-// Split-K plan for the FP8 x FP8 single-CTA plans when a workspace is
-// attached: if 128 x 128 tiles fill at most half of the SMs and K has at
-// least kSplitMinKBlocksTotal k-blocks, each tile is cut into S pieces of at
+// Split-K plan for the single-CTA plans of the FP8 linear and of the
+// weight-only linear when a workspace is attached: if 128 x 128 tiles fill at
+// most half of the SMs and K has at least kSplitMinKBlocksTotal k-blocks
+// (kSplitMinKBlocksTotalW8 of 64 elements for weight-only; each threshold is
+// a plain k-loop of ~13 us), each tile is cut into S pieces of at
 // least kSplitMinKBlocks k-blocks (S <= kSplitMaxPieces, tiles x S <= SMs), so
 // every CTA streams a short slice of W instead of one CTA per tile streaming
 // all of K. Returns S (1: no split).
 static int split_pieces(const fp8dit_linear* hs, int32_t n, int64_t M, int cfg, int num_sms) {
-    if ((cfg != kCfg128x128 && cfg != kCfg128x256 && cfg != kCfg128x64) || hs[0]->sk_ws == nullptr || M <= 0)
+    const bool wo = cfg == kCfgW8128x128;
+    if ((cfg != kCfg128x128 && cfg != kCfg128x256 && cfg != kCfg128x64 && !wo) || hs[0]->sk_ws == nullptr || M <= 0)
         return 1;
     int64_t tiles = 0;
     for (int g = 0; g < n; ++g) tiles += ((M + 127) / 128) * ((hs[g]->N + 127) / 128);
     if (tiles <= 0 || tiles * 2 > num_sms) return 1;
-    const int64_t num_kb = (hs[0]->K + 127) / 128;
-    if (num_kb < kSplitMinKBlocksTotal) return 1;
+    const int64_t ke = wo ? 64 : 128;  // K elements per k-block of the configuration
+    const int64_t num_kb = (hs[0]->K + ke - 1) / ke;
+    if (num_kb < (wo ? kSplitMinKBlocksTotalW8 : kSplitMinKBlocksTotal)) return 1;
+    // Weight-only at 33-128 rows and 32-63 k-blocks: the heavier reduction
+    // cancels the gain (measured: M = 128, K = 2048, 16.1 us plain vs 16.4 split).
+    if (wo && M > 64 && num_kb < 2 * kSplitMinKBlocksTotalW8) return 1;
     int64_t S = num_sms / tiles;
     if (S > num_kb / kSplitMinKBlocks) S = num_kb / kSplitMinKBlocks;
     if (S > kSplitMaxPieces) S = kSplitMaxPieces;
@@ -226,7 +233,7 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
                               uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev, int cfg,
                               const float* ra = nullptr) {
     const int split = split_pieces(hs, n, M, cfg, dev->num_sms);
-    if (split > 1) cfg = kCfg128x128;
+    if (split > 1 && !gemm_weight_only(cfg)) cfg = kCfg128x128;
     const int bm = gemm_block_m(cfg);
     const int bn = gemm_block_n(cfg);
     const int ke = gemm_k_elems(cfg);

@@ -122,7 +122,8 @@ struct alignas(64) GemmArgs {
     uint32_t* split_gen;     // split-K: generation word per tile (any value)
     uint32_t* sk_flag;   // stream-K: [units + 1][2 CTAs][8 epilogue warps] (zero between launches)
     float* sk_partial;   // stream-K: [units][2 CTAs][8 epilogue warps][32 rows][128 columns];
-                         // split-K: [tiles][split_k][4 quarters][2 halves][16 float4][32 rows]
+                         // split-K: [tiles][split_k][4 quarters][epilogue warps / 4 column parts]
+                         //          [128 / (epilogue warps / 4) / 4 float4][32 rows]
 };
 
 // Stream-K / split-K workspace for `units` CTA pairs: a flag area, then the
@@ -143,7 +144,8 @@ constexpr int64_t kSkMinKBlocks = 8;  // shorter tiles gain less from a split th
 // the split's fixed cost (~3.5 us: partial stores, the arrival handshake
 // across the GPU, the reduction). Measured: K = 8192 (64 k-blocks) runs 2.1x
 // faster at M <= 26 and 1.55x at M = 128; K = 2048 gains nothing.
-constexpr int kSplitMinKBlocksTotal = 48;  // split-K: k-blocks of the layer, at least
+constexpr int kSplitMinKBlocksTotal = 48;  // split-K: k-blocks of the layer, at least (FP8, 128 per block)
+constexpr int kSplitMinKBlocksTotalW8 = 32;  // the same for weight-only (64 bf16 per block: ~13 us plain)
 constexpr int kSplitMinKBlocks = 6;        // split-K: k-blocks per piece (one ring), at least
 constexpr int kSplitMaxPieces = 8;         // split-K: pieces per tile, at most
 constexpr size_t kSplitPieceBytes = 128 * 128 * sizeof(float);  // one fp32 128 x 128 partial

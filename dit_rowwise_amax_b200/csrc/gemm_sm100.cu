@@ -89,8 +89,10 @@ struct Cfg {
     static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
     static constexpr int EPI_WARPS = CONV ? 4 : 8;   // one or two per TMEM lane quarter
-    // Split-K is compiled only into the FP8 128 x 128 single-CTA kernel.
-    static constexpr bool SPLIT_OK = CG == 1 && BN == 128 && OPS == kOpsFp8;
+    // Split-K is compiled only into the 128 x 128 single-CTA kernels of the FP8
+    // linear and of the weight-only linear.
+    static constexpr bool SPLIT_OK = CG == 1 && BN == 128 && (OPS == kOpsFp8 || OPS == kOpsW8);
+    static constexpr int HALVES = EPI_WARPS / 4;  // epilogue warps per TMEM lane quarter
     static constexpr int CONV_WARPS = CONV ? STAGES : 0;  // converter warps, one per ring stage
     static constexpr int EPI_COLS = BN / (EPI_WARPS / 4);  // columns per epilogue warp
     static constexpr int BOX = 32;                   // epilogue store box: 32 rows x 32 columns
@@ -479,8 +481,9 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 const int r = ra + i / F4;
                 const int f = i % F4;
                 if (4 * f >= cols) continue;
-                // Partial layout of a piece: [quarter q][column half h][chunk float4 cv][row lane].
-                const int off = ((((r >> 5) * 2 + f / (C::EPI_COLS / 4)) * (C::EPI_COLS / 4) + f % (C::EPI_COLS / 4)) << 5) + (r & 31);
+                // Partial layout of a piece: [quarter q][column part h][float4 cv][row lane].
+                const int off = ((((r >> 5) * C::HALVES + f / (C::EPI_COLS / 4)) * (C::EPI_COLS / 4) +
+                                  f % (C::EPI_COLS / 4)) << 5) + (r & 31);
                 // Pieces in groups of four loads in flight, added in piece order.
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -599,13 +602,13 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 tmem_ld_32x32b_x32(t_addr + c * 32, r);
                 tmem_wait_ld();
                 if (split) {
-                    // This piece's raw fp32 partial, [q][half][chunk float4][lane]:
+                    // This piece's raw fp32 partial, [q][column part][float4][lane]:
                     // every warp store moves 512 contiguous bytes. Warps whose
                     // rows all lie past M store nothing (nothing reads them).
                     if (row0 < args.M) {
                         float4* dst = reinterpret_cast<float4*>(args.sk_partial) +
                                       (size_t)((int64_t)sg.t * args.split_k + sg.piece) * (C::ROWS * BN / 4) +
-                                      ((((size_t)q * 2 + (ew >> 2)) * (C::EPI_COLS / 4) + c * 8) << 5) + lane;
+                                      ((((size_t)q * C::HALVES + (ew >> 2)) * (C::EPI_COLS / 4) + c * 8) << 5) + lane;
 #pragma unroll
                         for (int v = 0; v < 8; ++v)
                             __stcg(dst + v * 32,

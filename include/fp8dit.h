@@ -183,11 +183,13 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  * fp32) but differ in rounding from the plain schedule.
  * The same workspace enables split-K for few tiles and a long K: when the
  * 128 x 128 tiles of a small-M call fill at most half of the SMs and K has at
- * least 48 k-blocks (K >= 6144; e.g. text tokens through an FFN-down weight),
- * each tile is cut into up to 8 pieces of at least 6 k-blocks on separate
- * CTAs; the pieces' fp32 partials are added in piece order (deterministic,
- * rounding differs from the plain schedule). fp8_scaled_linear_multi uses the
- * workspace of its first layer. Without a workspace, or for other shapes (the
+ * least 48 k-blocks of 128 (K >= 6144; e.g. text tokens through an FFN-down
+ * weight), each tile is cut into up to 8 pieces of at least 6 k-blocks on
+ * separate CTAs; the pieces' fp32 partials are added in piece order
+ * (deterministic, rounding differs from the plain schedule).
+ * fp8_weight_only_linear splits the same way from 32 k-blocks of 64 (K >=
+ * 2048; K >= 4096 above 64 rows). fp8_scaled_linear_multi uses the workspace
+ * of its first layer. Without a workspace, or for other shapes (the
  * FFN shapes among them), the plain schedule is used.
  *   fp8_linear_workspace_size: bytes needed on the layer's device (~19 MB on
  *     148 SMs), the same for every M.

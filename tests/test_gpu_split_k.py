@@ -157,7 +157,7 @@ def test_split_k_leaves_other_plans_alone(M, N, K):
 
 def test_one_workspace_for_mixed_plans():
     """One workspace shared, in stream order, by split-K launches of 16 and of 48
-    tiles and by stream-K launches (152 pair tiles), in an order where each
+    tiles (FP8 and weight-only) and by stream-K launches (152 pair tiles), in an order where each
     plan follows the others: every result equals the same layer's result on a
     workspace of its own, bit for bit, and no bounded wait expires. (The
     split-K counters and the stream-K flags occupy separate, fixed regions.)"""
@@ -170,20 +170,59 @@ def test_one_workspace_for_mixed_plans():
     lsk, _, _ = layer_and_codes(Wsk, synth.normal_bf16("gpu/split/mixed/bsk", (2048,), 0.1))
     a_small = fp8.quantize_rowwise(to_device_bf16(synth.normal_bf16("gpu/split/mixed/A", (26, K), 1.0)))
     a_sk = fp8.quantize_rowwise(to_device_bf16(synth.normal_bf16("gpu/split/mixed/Ask", (4800, 1040), 1.0)))
-    runs = {"16": (l16, a_small), "48": (l48, a_small), "sk": (lsk, a_sk)}
+    a_bf16 = to_device_bf16(synth.normal_bf16("gpu/split/mixed/Awo", (26, K), 1.0))
+    runs = {"16": (l16, a_small), "48": (l48, a_small), "sk": (lsk, a_sk), "wo": (l48, a_bf16)}
+
+    def call(name):
+        layer, arg = runs[name]
+        return layer.forward_weight_only(arg) if name == "wo" else layer.forward_fp8(*arg)
+
     ref = {}
-    for name, (layer, (qa, sa)) in runs.items():
+    for name, (layer, _) in runs.items():
+        torch.cuda.synchronize()  # attach only while no call of the layer is in flight
         layer.attach_workspace()  # a private workspace
-        ref[name] = layer.forward_fp8(qa, sa)
+        ref[name] = call(name)
     torch.cuda.synchronize()
     assert fp8.device_error() == 0
     assert l16.plan(26)[2] > 16 and l48.plan(26)[2] > 48  # both split
+    torch.cuda.synchronize()
     ws = l16.attach_workspace()
     l48.attach_workspace(ws)
     lsk.attach_workspace(ws)
-    for name in ["16", "48", "16", "sk", "48", "sk", "16", "48"]:
-        layer, (qa, sa) = runs[name]
-        y = layer.forward_fp8(qa, sa)
+    for name in ["16", "48", "wo", "16", "sk", "48", "wo", "sk", "16", "48"]:
+        y = call(name)
         torch.cuda.synchronize()
         assert fp8.device_error() == 0, f"a bounded wait expired in the {name} launch"
         assert torch.equal(y.view(torch.int16), ref[name].view(torch.int16)), name
+
+
+# FP8 weight-only linear (bf16 activation, E4M3 weight decoded in shared
+# memory): the same split with 64-element k-blocks, from 32 k-blocks on (64
+# above 64 rows). Ragged N and K at M = 60: 33 k-blocks, the last 16 elements.
+@pytest.mark.parametrize("M,N,K", [(1, 2048, 2048), (26, 2048, 8192), (60, 264, 2064), (128, 2048, 4096)])
+def test_weight_only_split_k(M, N, K):
+    A = synth.normal_bf16(f"gpu/split/wo/A/{M}x{K}", (M, K), 1.0, outlier_p=0.01, outlier_factor=20.0)
+    W = synth.normal_bf16(f"gpu/split/wo/W/{N}x{K}", (N, K), 0.02)
+    bias = synth.normal_bf16(f"gpu/split/wo/b/{N}", (N,), 0.1)
+    layer, qw, sw = layer_and_codes(W, bias)
+    a = to_device_bf16(A)
+    y_plain = layer.forward_weight_only(a)
+    layer.attach_workspace()
+    nbytes = M * N * 2
+    buf, view = canary_buffer(nbytes)
+    y1 = view.view(torch.bfloat16).view(M, N)
+    layer.forward_weight_only(a, y=y1)
+    y2 = layer.forward_weight_only(a)
+    torch.cuda.synchronize()
+    assert fp8.device_error() == 0
+    check_canary(buf, nbytes)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), "split-K result changed between runs"
+    ref = oracle.linear_weight_only(A, qw, sw, bias)
+    ok, worst = oracle.tolerance_ok(bf16_tensor_to_f64(y1), ref)
+    assert ok, f"tolerance exceeded: worst error / bound = {worst:.3f}"
+    if K >= 8192:  # tens of thousands of outputs: a different summation split shows in some bits
+        assert not torch.equal(y1.view(torch.int16), y_plain.view(torch.int16)), "no tile was split"
+    layer.detach_workspace()
+    y3 = layer.forward_weight_only(a)
+    torch.cuda.synchronize()
+    assert torch.equal(y3.view(torch.int16), y_plain.view(torch.int16))
