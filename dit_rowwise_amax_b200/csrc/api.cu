@@ -210,8 +210,9 @@ static int split_pieces(const fp8dit_linear* hs, int32_t n, int64_t M, int cfg, 
     const int64_t ke = wo ? 64 : 128;  // K elements per k-block of the configuration
     const int64_t num_kb = (hs[0]->K + ke - 1) / ke;
     if (num_kb < (wo ? kSplitMinKBlocksTotalW8 : kSplitMinKBlocksTotal)) return 1;
-    // Weight-only at 33-128 rows and 32-63 k-blocks: the heavier reduction
-    // cancels the gain (measured: M = 128, K = 2048, 16.1 us plain vs 16.4 split).
+    // Weight-only above 64 rows with fewer than 64 k-blocks: the heavier
+    // reduction cancels the gain (measured: M = 128, K = 2048, 16.1 us plain vs
+    // 16.4 split).
     if (wo && M > 64 && num_kb < 2 * kSplitMinKBlocksTotalW8) return 1;
     int64_t S = num_sms / tiles;
     if (S > num_kb / kSplitMinKBlocks) S = num_kb / kSplitMinKBlocks;
