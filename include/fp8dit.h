@@ -327,7 +327,11 @@ fp8dit_status fp8_scaled_linear_noalloc(fp8dit_linear h, int64_t M, const uint16
  * then all n products run in one grouped launch.
  *   hs  HOST array of n handles (1 <= n <= 4), all with the same K and device.
  *   ys  HOST array of n device pointers, ys[i] is [M, N_i] bf16.
- * Results are bitwise identical to n fp8_scaled_linear calls.
+ * Results are bitwise identical to n fp8_scaled_linear calls whenever the
+ * grouped launch and the single calls use the same tile plan and no split
+ * (e.g. the 256 x 256 pair plan of the hidden_states projections); a split
+ * schedule (workspace attached) may cut the grouped launch's K differently
+ * from a single call's and round differently, within the same bound.
  */
 fp8dit_status fp8_scaled_linear_multi(const fp8dit_linear* hs, int32_t n, int64_t M,
                                       const uint16_t* a_bf16, uint8_t* qa_scratch,
