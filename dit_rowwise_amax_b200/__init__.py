@@ -324,10 +324,12 @@ class FP8Linear:
             pass
 
     def attach_workspace(self, workspace: Optional[torch.Tensor] = None) -> Optional[torch.Tensor]:
-        """Attach a stream-K workspace (allocated here when not given) and
-        return it, so that it can be attached to further layers whose calls
-        run one after another; detach_workspace() goes back to the plain
-        schedule."""
+        """Attach a workspace (allocated here when not given) and return it,
+        so that it can be attached to further layers whose calls run one after
+        another. It enables the stream-K schedule (a nearly empty last wave of
+        pair tiles) and split-K (few rows and a long K, FP8 and weight-only);
+        detach_workspace() goes back to the plain schedule. Attach only while
+        no call of the layer is in flight."""
         L = load_library()
         need = int(L.fp8_linear_workspace_size(self._h))
         if workspace is None:
