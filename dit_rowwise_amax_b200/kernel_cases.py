@@ -12,6 +12,8 @@ Cases (inputs from ``synth``, the same as the benchmark's):
     fused_ffn_up, fused_ffn_down         quantise-in-GEMM variant (row-scale pre-pass + GEMM)
     gemm_text_ffn_down                   FP8 GEMM, 26 tokens x FFN-down weight, plain schedule
     split_k_text_ffn_down                the same with a workspace attached (split-K schedule)
+    weight_only_text_ffn_down            FP8 weight-only GEMM, 26 tokens x FFN-down weight
+    split_k_weight_only_text_ffn_down    the same with a workspace attached (split-K schedule)
     state_dict_e4m3fn, state_dict_e5m2   per-tensor conversion of the 192-tensor DiT weight set
 Layer creation runs the per-channel weight quantiser first; every case then
 launches only its own kernels. Exits non-zero if the device reports an error.
@@ -28,7 +30,8 @@ from . import E4M3FN, E5M2, FP8Linear, act_quantize_rowwise, device_error, quant
 
 CASES = ("quantize_ffn_up", "quantize_ffn_down", "quantize_hidden", "gelu_quantize_ffn_down", "gemm_ffn_up", "gemm_ffn_down",
          "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down", "gemm_text_ffn_down",
-         "split_k_text_ffn_down", "state_dict_e4m3fn", "state_dict_e5m2")
+         "split_k_text_ffn_down", "weight_only_text_ffn_down", "split_k_weight_only_text_ffn_down",
+         "state_dict_e4m3fn", "state_dict_e5m2")
 TEXT_TOKENS = 26  # encoder_hidden_states length
 
 
@@ -69,13 +72,14 @@ def run(case: str, iters: int) -> None:
     else:
         layer = FP8Linear.from_weight(_dev(workload["W"], dev), _dev(workload["bias"], dev))
         y = torch.empty((M, layer.N), dtype=torch.bfloat16, device=dev)
-        if case.startswith("split_k"):
+        op = case[len("split_k_"):] if case.startswith("split_k_") else case
+        if op != case:
             layer.attach_workspace()
-        if case.startswith("gemm") or case.startswith("split_k"):
+        if op.startswith("gemm") or op == "text_ffn_down":
             qa, sa = quantize_rowwise(a)
             for _ in range(iters):
                 layer.forward_fp8(qa, sa, y=y)
-        elif case.startswith("weight_only"):
+        elif op.startswith("weight_only"):
             for _ in range(iters):
                 layer.forward_weight_only(a, y=y)
         else:
