@@ -350,6 +350,10 @@ class FP8Linear:
                                               ctypes.byref(ctas)))
         return bm.value, bn.value, ctas.value
 
+    def __call__(self, a: torch.Tensor, **kwargs) -> torch.Tensor:
+        """layer(a) is layer.forward(a): quantise + FP8 GEMM + epilogue."""
+        return self.forward(a, **kwargs)
+
     def forward(self, a: torch.Tensor, y: Optional[torch.Tensor] = None,
                 qa_scratch: Optional[torch.Tensor] = None,
                 sa_scratch: Optional[torch.Tensor] = None) -> torch.Tensor:

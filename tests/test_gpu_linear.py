@@ -53,6 +53,9 @@ def test_tiny_config_full():
     layer, qw, sw = make_layer(d["W"], d["bias"])
     y, qa, sa = run_bf16(layer, d["A"])
     check_full(y, qa, sa, qw, sw, d["bias"])
+    y_call = layer(to_device_bf16(d["A"]))  # the layer is callable like a torch module
+    torch.cuda.synchronize()
+    assert torch.equal(y_call.view(torch.int16), y.view(torch.int16))
 
 
 def test_ffn_up_full_size():
