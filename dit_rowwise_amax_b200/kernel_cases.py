@@ -15,6 +15,8 @@ Cases (inputs from ``synth``, the same as the benchmark's):
     weight_only_text_ffn_down            FP8 weight-only GEMM, 26 tokens x FFN-down weight
     split_k_weight_only_text_ffn_down    the same with a workspace attached (split-K schedule)
     state_dict_e4m3fn, state_dict_e5m2   per-tensor conversion of the 192-tensor DiT weight set
+    qkv_encoder                          Q/K/V projections of encoder_hidden_states [26, 2048]:
+                                         one quantise + one grouped GEMM (128 x 64 tiles)
     state_dict_e4m3fn_4blocks            the same on the first 4 blocks' 24 tensors (400 MB of bf16,
                                          above L2; small enough for a multi-pass profile)
 Layer creation runs the per-channel weight quantiser first; every case then
@@ -28,12 +30,13 @@ import torch
 
 import synth
 
-from . import E4M3FN, E5M2, FP8Linear, act_quantize_rowwise, device_error, quantize_per_tensor, quantize_rowwise
+from . import (E4M3FN, E5M2, FP8Linear, act_quantize_rowwise, device_error, quantize_per_tensor, quantize_rowwise,
+               scaled_linear_multi)
 
 CASES = ("quantize_ffn_up", "quantize_ffn_down", "quantize_hidden", "gelu_quantize_ffn_down", "gemm_ffn_up", "gemm_ffn_down",
          "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down", "gemm_text_ffn_down",
          "split_k_text_ffn_down", "weight_only_text_ffn_down", "split_k_weight_only_text_ffn_down",
-         "state_dict_e4m3fn", "state_dict_e5m2", "state_dict_e4m3fn_4blocks")
+         "state_dict_e4m3fn", "state_dict_e5m2", "state_dict_e4m3fn_4blocks", "qkv_encoder")
 STATE_DICT_4BLOCKS = 24  # tensors in the first four DiT blocks
 TEXT_TOKENS = 26  # encoder_hidden_states length
 
@@ -54,6 +57,20 @@ def run(case: str, iters: int) -> None:
         fmt = E5M2 if "e5m2" in case else E4M3FN
         for _ in range(iters):
             quantize_per_tensor(tensors, fmt, outs=outs, scales=scales)
+        torch.cuda.synchronize()
+        if device_error() != 0:
+            raise SystemExit(f"{case}: device error word set")
+        return
+    if case == "qkv_encoder":
+        att = synth.attention()
+        layers = [FP8Linear.from_weight(_dev(att[f"W_{p}"], dev), _dev(att[f"bias_{p}"], dev)) for p in "qkv"]
+        a = _dev(att["encoder"], dev)
+        M, K = a.shape
+        qa = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        sa = torch.empty((M,), dtype=torch.float32, device=dev)
+        ys = [torch.empty((M, layer.N), dtype=torch.bfloat16, device=dev) for layer in layers]
+        for _ in range(iters):
+            scaled_linear_multi(layers, a, ys=ys, qa_scratch=qa, sa_scratch=sa)
         torch.cuda.synchronize()
         if device_error() != 0:
             raise SystemExit(f"{case}: device error word set")
