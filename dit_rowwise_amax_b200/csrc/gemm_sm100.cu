@@ -2,10 +2,10 @@
 // and bf16 epilogue, for sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
 // What it computes ("从 BF16 到 FP8：HunyuanVideo1.5推理优化复盘", section 三.1,
-// the "FP8 GEMM -> scale / bias / output dtype" steps, and section 三.2 item 4:
+// the steps after the FP8 GEMM: scales, bias, output type; section 三.2 item 4:
 // the full path with bias, scale and output dtype, not a bare GEMM):
 //     y[m, n] = bf16_rne( (sum_k A[m,k] W[n,k]) * sa[m] * sw[n] + bias[n] )
-// A [M, K] and W [N, K] are both K-major (the "column-major B" of section 三.1,
+// A [M, K] and W [N, K] are both K-major (section 三.1's column-major B operand,
 // fixed at weight preparation, so no transpose ever reaches this kernel).
 //
 // Structure (persistent over output tiles, one CTA per SM):

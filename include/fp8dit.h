@@ -225,8 +225,8 @@ fp8dit_status fp8_scaled_linear(fp8dit_linear h, int64_t M, const uint16_t* a_bf
                                 float* sa_scratch, uint16_t* y, fp8dit_stream_t stream);
 
 /*
- * FP8 weight-only linear: the "FP8 weight-only scaled" pipeline the
- * longcat-avatar-compare page sets against NVFP4 W4A4 (section 速度总览). The
+ * FP8 weight-only linear: the FP8 weight-only configuration with scales that
+ * the longcat-avatar-compare page sets against NVFP4 W4A4 (section 速度总览). The
  * activation is not quantised; the layer's E4M3 weight is decoded to bf16 in
  * shared memory and multiplied on the BF16 tensor cores:
  *   y[m, n] = bf16_rne( (sum_k A[m,k] dec(qw[n,k])) * sw[n] + bias[n] ), fp32 accumulation.

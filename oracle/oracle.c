@@ -209,8 +209,8 @@ void or_dot_units(const uint8_t* qa, const uint8_t* qw, int64_t M, int64_t N, in
 
 /* ----------------------------------------------------- FP8 weight-only linear */
 /*
- * The "FP8 weight-only scaled" pipeline compared on the longcat-avatar-compare
- * page (section 速度总览): the activation stays bf16, only the weight is FP8
+ * The FP8 weight-only configuration with scales, compared on the
+ * longcat-avatar-compare page (section 速度总览): the activation stays bf16, only the weight is FP8
  * with its per-channel scale.
  *   y[m, n] = (sum_k A[m,k] dec(qw[n,k])) * sw[n] + bias[n], in double.
  * Every product of a bf16 value (8 significant bits) and an E4M3 value (4) is
