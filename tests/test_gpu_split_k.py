@@ -226,3 +226,33 @@ def test_weight_only_split_k(M, N, K):
     y3 = layer.forward_weight_only(a)
     torch.cuda.synchronize()
     assert torch.equal(y3.view(torch.int16), y_plain.view(torch.int16))
+
+
+TIMEOUT = 5  # FP8DIT_ERR_TIMEOUT
+
+
+def test_split_k_expired_wait_reports_timeout():
+    """A split-K arrival that can never complete: the first tile's arrival
+    counter is planted far above the piece count (the kind of state an
+    interrupted launch leaves), so no piece sees the count it waits for. Each
+    piece's bounded wait expires (about 2 s), the host reads
+    FP8DIT_ERR_TIMEOUT, and after the workspace is attached again (which
+    clears its counters) the same call gives the normal result."""
+    M, N, K = 26, 2048, 8192
+    W = synth.normal_bf16(f"gpu/split/W/{N}x{K}", (N, K), 0.02)
+    layer, _, _ = layer_and_codes(W, synth.normal_bf16(f"gpu/split/b/{N}", (N,), 0.1))
+    ws = layer.attach_workspace()
+    qa, sa = fp8.quantize_rowwise(to_device_bf16(synth.normal_bf16("gpu/split/timeout/A", (M, K), 1.0)))
+    y_ref = layer.forward_fp8(qa, sa)
+    assert fp8.device_error() == 0
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    arrive0 = (pairs + 1) * 16  # first split-K arrival counter, in 32-bit words (after the stream-K flags)
+    ws.view(torch.int32)[arrive0] = 1 << 30
+    torch.cuda.synchronize()
+    layer.forward_fp8(qa, sa)
+    assert fp8.device_error() == TIMEOUT
+    assert fp8.device_error() == 0  # reading clears the word
+    layer.attach_workspace(ws)  # clears the counters
+    y = layer.forward_fp8(qa, sa)
+    assert fp8.device_error() == 0
+    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
