@@ -154,6 +154,7 @@ cudaError_t launch_selftest_wait(cudaStream_t stream, DevErr err) {
 using namespace fp8dit;
 
 int64_t fp8dit::linear_k(const fp8dit_linear_s* h) { return h->K; }
+int fp8dit::linear_device(const fp8dit_linear_s* h) { return h->device; }
 
 static int64_t tiles_for(const fp8dit_linear_s* h, int64_t M, int n_problems, int cfg) {
     const int64_t bm = gemm_block_m(cfg), bn = gemm_block_n(cfg);

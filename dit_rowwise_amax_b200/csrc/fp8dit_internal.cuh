@@ -40,8 +40,9 @@ const DeviceInfo* device_info();
 void set_error(const char* fmt, ...);
 fp8dit_status cuda_fail(cudaError_t e, const char* what);
 
-// Reduction length K of a linear layer handle.
+// Reduction length K and CUDA device of a linear layer handle.
 int64_t linear_k(const fp8dit_linear_s* h);
+int linear_device(const fp8dit_linear_s* h);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point: a 2-D
 // row-major tensor of 1- or 2-byte elements (inner = contiguous extent).

@@ -63,6 +63,7 @@ fp8dit_status scratch_address(uint8_t** out) {
 
 extern "C" fp8dit_status fp8_scaled_linear_noalloc(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, uint16_t* y,
                                                    fp8dit_stream_t stream) {
+    fp8dit::set_error("%s", "");
     if (!h) {
         fp8dit::set_error("invalid argument: null handle");
         return FP8DIT_ERR_INVALID_ARG;
@@ -81,6 +82,16 @@ extern "C" fp8dit_status fp8_scaled_linear_noalloc(fp8dit_linear h, int64_t M, c
         return FP8DIT_ERR_UNSUPPORTED_SHAPE;
     }
     if (M == 0) return FP8DIT_OK;
+    // The array's address is looked up on the current device, so that must be
+    // the layer's device (checked before the lookup, which would otherwise
+    // load the library's device image, array included, onto another GPU).
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fp8dit::cuda_fail(e, "cudaGetDevice");
+    if (dev != fp8dit::linear_device(h)) {
+        fp8dit::set_error("invalid argument: current device differs from the layer's device");
+        return FP8DIT_ERR_INVALID_ARG;
+    }
     uint8_t* scratch = nullptr;
     fp8dit_status st = scratch_address(&scratch);
     if (st != FP8DIT_OK) return st;

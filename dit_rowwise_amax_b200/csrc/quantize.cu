@@ -20,12 +20,15 @@
 //
 // Producer fusion ("从 BF16 到 FP8", section 三.5): with ACT != 0 the kernels
 // first replace each loaded element by bf16(act(x)) — GELU (erf or tanh form)
-// or SiLU, evaluated in fp32 with erfcf / expf in forms that do not cancel
-// for negative x — optionally store that bf16 tensor, and quantise it.
-// A bf16 input has only 65536 values, so bf16(act(x)) is evaluated once per
-// device for every bf16 pattern into a 128 KB table (act_table_kernel) and the
-// quantisers read the table: the same values, one cached load per element
-// instead of an erfc / exp evaluation.
+// or SiLU — optionally store that bf16 tensor, and quantise it. A bf16 input
+// has only 65536 values, so bf16(act(x)) is evaluated once per device for
+// every bf16 pattern into a 128 KB table (act_table_kernel) and the
+// quantisers read the table: one cached load per element. Since the table is
+// built once, each entry is evaluated in double (CUDA's double erfc / exp, in
+// forms that do not cancel for negative x, every other operation an
+// explicitly rounded IEEE double operation) and rounded once to bf16, ties to
+// even: the correctly rounded activation except where the true value lies
+// within a few double ulps of a bf16 rounding boundary.
 #include <algorithm>
 #include <mutex>
 
@@ -36,25 +39,42 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// x / (1 + exp(-t)) without overflow: for t < 0 it is x e^t / (1 + e^t).
-__device__ __forceinline__ float x_logistic(float x, float t) {
-    if (t >= 0.0f) return x / (1.0f + expf(-t));
-    const float e = expf(t);
-    return (x * e) / (1.0f + e);
-}
-
+// The activation in double. Every product, sum and quotient is an explicitly
+// rounded IEEE double operation (no contraction into FMAs), so the only
+// inexact steps besides them are CUDA's double erfc and exp:
+//   GELU, erf form    (x / 2) erfc(-x / sqrt 2)                 = x Phi(x)
+//   GELU, tanh form   x / (1 + exp(-2 sqrt(2/pi) (x + 0.044715 x^3)))
+//   SiLU              x / (1 + exp(-x))
+// The right-hand forms do not cancel for negative x (1 + erf and 1 + tanh
+// would). exp overflowing to +inf gives x / inf = -0 for very negative x.
 template <int ACT>
-__device__ __forceinline__ float act_f(float x) {
+__device__ double act_d(double x) {
     if constexpr (ACT == FP8DIT_ACT_GELU_ERF) {
-        return 0.5f * x * erfcf(-x * 0.70710678118654752f);  // x Phi(x)
+        return __dmul_rn(__dmul_rn(0.5, x), erfc(__ddiv_rn(-x, __dsqrt_rn(2.0))));
     } else if constexpr (ACT == FP8DIT_ACT_GELU_TANH) {
-        const float u = 0.79788456080286536f * (x + 0.044715f * x * x * x);
-        return x_logistic(x, 2.0f * u);  // x/2 (1 + tanh u)
+        const double c = __dmul_rn(-2.0, __dsqrt_rn(__ddiv_rn(2.0, 3.14159265358979323846)));
+        const double cube = __dmul_rn(__dmul_rn(__dmul_rn(0.044715, x), x), x);
+        return __ddiv_rn(x, __dadd_rn(1.0, exp(__dmul_rn(c, __dadd_rn(x, cube)))));
     } else if constexpr (ACT == FP8DIT_ACT_SILU) {
-        return x_logistic(x, x);
+        return __ddiv_rn(x, __dadd_rn(1.0, exp(-x)));
     } else {
         return x;
     }
+}
+
+// Nearest bf16 to a double, ties to even, in one rounding: truncate to fp32
+// and set the lowest bit when that dropped anything (round to odd; fp32 keeps
+// 16 more significand bits than bf16, subnormals included), then round that
+// fp32 to bf16 to nearest even. Rounding to odd with at least two extra bits
+// followed by round-to-nearest equals one round-to-nearest (Boldo and
+// Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms
+// using rounding to odd", IEEE Trans. Computers 57(4), 2008).
+__device__ __forceinline__ uint16_t bf16_rne_of_double(double v) {
+    const float f = __double2float_rz(v);
+    uint32_t u = __float_as_uint(f);
+    if ((double)f != v) u |= 1u;
+    const __nv_bfloat16 r = __float2bfloat16_rn(__uint_as_float(u));
+    return *reinterpret_cast<const uint16_t*>(&r);
 }
 
 // bf16(act(x)) for every bf16 pattern x, one table per activation.
@@ -64,8 +84,7 @@ template <int ACT>
 __global__ void act_table_kernel() {
     const uint32_t b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= 65536u) return;
-    const __nv_bfloat16 r = __float2bfloat16_rn(act_f<ACT>(__uint_as_float(b << 16)));
-    g_act_table[ACT - 1][b] = *reinterpret_cast<const uint16_t*>(&r);
+    g_act_table[ACT - 1][b] = bf16_rne_of_double(act_d<ACT>((double)__uint_as_float(b << 16)));
 }
 
 // bf16(act(x)) for the eight bf16 of a 16-byte vector.

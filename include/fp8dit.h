@@ -102,8 +102,10 @@ typedef enum {
  * FFN-down emits the (FP8 tensor, per-token scale) pair directly instead of a
  * bf16 tensor that a separate pass then quantises.
  *   h     [M, K] bf16 (the FFN-up output), row stride ldh elements (ldh % 8 == 0), 16-byte aligned.
- *   g     = bf16_rne(act(h)), evaluated in fp32 (CUDA erfcf / expf); stored to
- *         gout [M, K] (row stride ldg, 16-byte aligned) when gout != NULL.
+ *   g     = bf16_rne(act(h)): act evaluated in double (CUDA's double erfc / exp,
+ *         every other step an IEEE double operation) and rounded once to bf16,
+ *         ties to even; stored to gout [M, K] (row stride ldg, 16-byte aligned)
+ *         when gout != NULL.
  *   q, scale: the rowwise recipe applied to g, E4M3FN codes (the GEMM's input).
  * Same shape rules as fp8_quantize_rowwise. The first call on a device builds
  * a 128 KB table per activation (bf16(act(x)) for all 65536 bf16 x, in static

@@ -1,7 +1,7 @@
 """Run one kernel of the FP8 linear path a few times on the synthetic workload
 inputs, for profiling it on its own (for example under Nsight Compute):
 
-    python -m dit_rowwise_amax_b200.kernel_cases weight_only_ffn_up --iters 4
+    python kernel_cases.py weight_only_ffn_up --iters 4
 
 Cases (inputs from ``synth``, the same as the benchmark's):
     quantize_ffn_up, quantize_ffn_down   rowwise E4M3 quantiser on the FFN activations
@@ -23,15 +23,19 @@ Layer creation runs the per-channel weight quantiser first; every case then
 launches only its own kernels. Exits non-zero if the device reports an error.
 """
 import argparse
+import os
 import sys
 
-import numpy as np
-import torch
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
 
-import synth
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
 
-from . import (E4M3FN, E5M2, FP8Linear, act_quantize_rowwise, device_error, quantize_per_tensor, quantize_rowwise,
-               scaled_linear_multi)
+import synth  # noqa: E402
+from dit_rowwise_amax_b200 import (E4M3FN, E5M2, FP8Linear, act_quantize_rowwise, device_error,  # noqa: E402
+                                   quantize_per_tensor, quantize_rowwise, scaled_linear_multi)
 
 CASES = ("quantize_ffn_up", "quantize_ffn_down", "quantize_hidden", "gelu_quantize_ffn_down", "gemm_ffn_up", "gemm_ffn_down",
          "weight_only_ffn_up", "weight_only_ffn_down", "fused_ffn_up", "fused_ffn_down", "gemm_text_ffn_down",

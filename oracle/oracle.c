@@ -37,6 +37,7 @@
 #include <math.h>
 #include <omp.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 enum { OR_E4M3FN = 0, OR_E5M2 = 1 };
@@ -223,15 +224,21 @@ void or_linear_weight_only(const uint16_t* a, const uint8_t* qw, const float* sw
         double v = or_decode(OR_E4M3FN, (uint8_t)c);
         wv[c] = isnan(v) ? 0.0 : v;
     }
-#pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t m = 0; m < M; ++m) {
-        for (int64_t n = 0; n < N; ++n) {
-            double dot = 0.0;
-            for (int64_t k = 0; k < K; ++k) dot += (double)or_bf16_to_f32(a[m * K + k]) * wv[qw[n * K + k]];
-            double v = dot * (double)sw[n];
-            if (bias) v += (double)or_bf16_to_f32(bias[n]);
-            y[m * N + n] = v;
+#pragma omp parallel
+    {
+        double* arow = (double*)malloc((size_t)K * sizeof(double)); /* row m of A as doubles (exact) */
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t m = 0; m < M; ++m) {
+            for (int64_t k = 0; k < K; ++k) arow[k] = (double)or_bf16_to_f32(a[m * K + k]);
+            for (int64_t n = 0; n < N; ++n) {
+                double dot = 0.0;
+                for (int64_t k = 0; k < K; ++k) dot += arow[k] * wv[qw[n * K + k]];
+                double v = dot * (double)sw[n];
+                if (bias) v += (double)or_bf16_to_f32(bias[n]);
+                y[m * N + n] = v;
+            }
         }
+        free(arow);
     }
 }
 

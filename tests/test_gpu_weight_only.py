@@ -31,14 +31,12 @@ def check_rows(y, A, qw, sw, bias, rows):
 
 @pytest.mark.parametrize("cfg", ["ffn_up", "ffn_down"])
 def test_ffn_full_size(cfg):
+    """Every output of both FFN layers (4096 rows, the 256 x 256 pair plan)."""
     d = getattr(synth, cfg)()
     layer, qw, sw = make_layer(d["W"], d["bias"])
     y = layer.forward_weight_only(to_device_bf16(d["A"]))
     torch.cuda.synchronize()
-    M = d["A"].shape[0]
-    rng = np.random.default_rng(1)
-    rows = np.unique(np.concatenate([np.arange(40), np.arange(M - 40, M), rng.integers(0, M, 24)]))
-    check_rows(y, d["A"], qw, sw, d["bias"], rows)
+    check_rows(y, d["A"], qw, sw, d["bias"], np.arange(d["A"].shape[0]))
 
 
 def test_tiny_config_full():
