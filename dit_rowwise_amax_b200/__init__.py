@@ -50,7 +50,12 @@ def library_path() -> str:
 
 class _TensorDesc(ctypes.Structure):
     _fields_ = [("src", ctypes.c_void_p), ("numel", ctypes.c_int64), ("dst", ctypes.c_void_p),
-                ("scale", ctypes.c_void_p)]
+                ("scale", ctypes.c_void_p), ("src_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+# Source element types of the per-tensor conversion (fp8dit_src_dtype).
+_SRC_DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+_FP8_DTYPES = (torch.float8_e4m3fn, torch.float8_e5m2)
 
 
 def load_library():
@@ -211,11 +216,21 @@ def quantize_weight_per_channel(w: torch.Tensor, fmt=E4M3FN) -> Tuple[torch.Tens
     return qw, sw
 
 
+def _src_dtype(t: torch.Tensor) -> int:
+    if t.dtype in (torch.int16, torch.uint16):  # raw bf16 bit patterns
+        return 0
+    try:
+        return _SRC_DTYPES[t.dtype]
+    except KeyError:
+        raise ValueError(f"tensors must be bfloat16, float16 or float32 (got {t.dtype})") from None
+
+
 def quantize_per_tensor(tensors: Sequence[torch.Tensor], fmt=E5M2,
                         outs: Optional[Sequence[torch.Tensor]] = None,
                         scales: Optional[torch.Tensor] = None,
                         workspace: Optional[torch.Tensor] = None) -> Tuple[List[torch.Tensor], torch.Tensor]:
-    """Per-tensor amax conversion of bf16 tensors -> (codes uint8 per tensor, S float32 [n])."""
+    """Per-tensor amax conversion of bf16 / fp16 / fp32 tensors (dtypes may be
+    mixed) -> (codes uint8 per tensor, S float32 [n])."""
     L = load_library()
     n = len(tensors)
     if n == 0:
@@ -224,8 +239,7 @@ def quantize_per_tensor(tensors: Sequence[torch.Tensor], fmt=E5M2,
     for t in tensors:
         if not t.is_cuda or t.device != dev or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors on one device")
-        if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
-            raise ValueError(f"tensors must hold bf16 values (got {t.dtype})")
+        _src_dtype(t)
     if outs is None:
         outs = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in tensors]
     if scales is None:
@@ -244,25 +258,37 @@ def quantize_per_tensor(tensors: Sequence[torch.Tensor], fmt=E5M2,
     for i, (t, o) in enumerate(zip(tensors, outs)):
         descs[i].src, descs[i].numel, descs[i].dst = t.data_ptr(), t.numel(), o.data_ptr()
         descs[i].scale = scales.data_ptr() + 4 * i
+        descs[i].src_dtype, descs[i].reserved = _src_dtype(t), 0
     _check(L.fp8_quantize_weight_per_tensor(descs, n, _fmt(fmt), workspace.data_ptr(),
                                             workspace.numel() * workspace.element_size(), _stream(dev)))
     return list(outs), scales
 
 
 def convert_state_dict(state_dict, fp8_format: str = "float8_e5m2"):
-    """Convert a state-dict's bf16 tensors to FP8 with one amax scale each
+    """Convert a state-dict's floating tensors to FP8 with one amax scale each
     ("Quantize Model to FP8 Format": model_state_dict + fp8_format, default
     float8_e5m2). Returns (quantised dict, {name: fp32 scale tensor}).
 
-    bf16 CUDA tensors with numel > 0 are converted; every other entry passes
-    through unchanged. Raises ValueError("Invalid input.") for a non-dict or
-    empty dict, and Fp8DitError (EMPTY) when no tensor was converted.
+    bfloat16, float16 and float32 tensors with numel > 0 are converted, in one
+    launch whatever the mix of dtypes; they must be on a CUDA device (there is
+    no CPU path). Non-floating entries, empty tensors and tensors that are
+    already FP8 pass through unchanged. Any other floating dtype (float64)
+    raises ValueError rather than passing through unconverted. Raises
+    ValueError("Invalid input.") for a non-dict or empty dict, and Fp8DitError
+    (EMPTY) when no tensor was converted.
     """
     if not isinstance(state_dict, dict) or len(state_dict) == 0:
         raise ValueError("Invalid input.")
     fmt = _fmt(fp8_format)
-    names = [k for k, v in state_dict.items()
-             if isinstance(v, torch.Tensor) and v.is_cuda and v.dtype == torch.bfloat16 and v.numel() > 0]
+    names = []
+    for k, v in state_dict.items():
+        if not isinstance(v, torch.Tensor) or not v.is_floating_point() or v.dtype in _FP8_DTYPES or v.numel() == 0:
+            continue
+        if v.dtype not in _SRC_DTYPES:
+            raise ValueError(f"{k}: {v.dtype} is not convertible (bfloat16, float16 or float32)")
+        if not v.is_cuda:
+            raise ValueError(f"{k}: floating tensors must be on a CUDA device to be converted")
+        names.append(k)
     if not names:
         raise Fp8DitError(3, f"No tensor converted to {fp8_format}.")
     tensors = [state_dict[k].contiguous() for k in names]

@@ -402,6 +402,9 @@ fp8dit_status fp8_quantize_weight_per_tensor(const fp8dit_tensor_desc* tensors, 
     for (int32_t i = 0; i < n_tensors; ++i) {
         const fp8dit_tensor_desc& d = tensors[i];
         if (d.numel < 0) return invalid("numel must be >= 0");
+        if (d.src_dtype != FP8DIT_SRC_BF16 && d.src_dtype != FP8DIT_SRC_F16 && d.src_dtype != FP8DIT_SRC_F32)
+            return invalid("src_dtype must be FP8DIT_SRC_BF16, FP8DIT_SRC_F16 or FP8DIT_SRC_F32");
+        if (d.reserved != 0) return invalid("reserved must be 0");
         if (d.numel == 0) continue;
         if (d.numel > ((int64_t)1 << 40)) return unsupported("tensor too large");
         if (!d.src || !d.dst || !d.scale) return invalid("null pointer in tensor descriptor");

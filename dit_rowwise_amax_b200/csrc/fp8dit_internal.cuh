@@ -64,10 +64,11 @@ cudaError_t launch_act_quantize_rows(const uint16_t* h, int64_t M, int64_t K, in
                                      const DeviceInfo* dev);
 
 struct PerTensorDevDesc {
-    const uint16_t* src;
+    const void* src;
     int64_t numel;
     uint8_t* dst;
     float* scale;
+    int32_t src_dtype;  // fp8dit_src_dtype
 };
 size_t per_tensor_workspace_bytes(int32_t n);
 cudaError_t launch_per_tensor(const fp8dit_tensor_desc* host_descs, int32_t n, int fmt, void* ws,

@@ -14,6 +14,8 @@
 // are done. Chunks are claimed in queue order by running blocks, and amax
 // chunks never wait, so every wait is on work already held by a running
 // block: the launch cannot deadlock whatever the grid size.
+#include <cuda_fp16.h>
+
 #include <algorithm>
 
 #include "fp8_codec.cuh"
@@ -24,7 +26,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kBatch = 192;              // tensors per launch (descriptors travel as kernel parameters)
 constexpr int64_t kChunk = 32768;        // elements per work item
-constexpr int kVecPerThread = kChunk / 8 / kThreads;  // 16 vectors of 8 bf16
 
 struct PerTensorArgs {
     PerTensorDevDesc d[kBatch];
@@ -44,6 +45,157 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
 }
 __device__ __forceinline__ void red_add_release_gpu(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---- source element types. A 16-byte vector holds 8 bf16 / fp16 values or
+// 4 fp32 values; the amax is kept as the bit pattern of |x| in the source
+// type (for non-negative values bit-pattern order is value order).
+template <int SRC>
+struct Src {
+    static constexpr int kEpv = SRC == FP8DIT_SRC_F32 ? 4 : 8;  // elements per 16-byte vector
+};
+
+template <int SRC>
+__device__ __forceinline__ float abs_bits_to_float(uint32_t bits) {
+    if constexpr (SRC == FP8DIT_SRC_BF16) return bf16_bits_to_float(bits);
+    else if constexpr (SRC == FP8DIT_SRC_F16) return __half2float(__ushort_as_half((unsigned short)bits));
+    else return __uint_as_float(bits);
+}
+
+// |x| bits of element e (tails).
+template <int SRC>
+__device__ __forceinline__ uint32_t abs_bits1(const void* src, int64_t e) {
+    if constexpr (SRC == FP8DIT_SRC_F32) return __float_as_uint(static_cast<const float*>(src)[e]) & 0x7fffffffu;
+    else return (uint32_t)static_cast<const uint16_t*>(src)[e] & 0x7fffu;
+}
+
+// Running max of |x| over a vector: packed pairs for the 16-bit types (folded
+// by the caller), one word for fp32.
+template <int SRC>
+__device__ __forceinline__ uint32_t absmax_vec(const uint4& v, uint32_t acc) {
+    if constexpr (SRC == FP8DIT_SRC_BF16) {
+        return absmax8(v, acc);
+    } else if constexpr (SRC == FP8DIT_SRC_F16) {
+        acc = __vmaxu2(acc, v.x & 0x7fff7fffu);
+        acc = __vmaxu2(acc, v.y & 0x7fff7fffu);
+        acc = __vmaxu2(acc, v.z & 0x7fff7fffu);
+        return __vmaxu2(acc, v.w & 0x7fff7fffu);
+    } else {
+        acc = max(acc, v.x & 0x7fffffffu);
+        acc = max(acc, v.y & 0x7fffffffu);
+        acc = max(acc, v.z & 0x7fffffffu);
+        return max(acc, v.w & 0x7fffffffu);
+    }
+}
+
+// FP8 codes of two fp32 values divided by s (IEEE division), low element first.
+template <int FMT>
+__device__ __forceinline__ uint32_t codes2_div(float lo, float hi, float s) {
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(lo, s), __fdiv_rn(hi, s)), __NV_SATFINITE,
+                                              Fp8Fmt<FMT>::kInterp);
+}
+
+// fp16 / fp32 sources: one vector -> its codes (8 bytes for fp16, 4 for fp32,
+// as the low bytes of a uint2). Every quotient is the IEEE division x / S (the
+// corrected-reciprocal quotient of the bf16 kernels is proven for bf16 inputs
+// only); each code takes its sign bit from x.
+template <int SRC, int FMT>
+__device__ __forceinline__ uint2 quant_vec_div(const uint4& v, float s) {
+    if constexpr (SRC == FP8DIT_SRC_F16) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t c[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+            c[k] = codes2_div<FMT>(f.x, f.y, s);
+        }
+        return make_uint2((c[0] | (c[1] << 16)) | signs4(w[0], w[1]), (c[2] | (c[3] << 16)) | signs4(w[2], w[3]));
+    } else {
+        const uint32_t c = codes2_div<FMT>(__uint_as_float(v.x), __uint_as_float(v.y), s) |
+                           (codes2_div<FMT>(__uint_as_float(v.z), __uint_as_float(v.w), s) << 16);
+        const uint32_t signs = ((v.x >> 24) & 0x80u) | ((v.y >> 16) & 0x8000u) | ((v.z >> 8) & 0x800000u) |
+                               (v.w & 0x80000000u);
+        return make_uint2(c | signs, 0u);
+    }
+}
+
+// One element -> its code (tails), for any source type.
+template <int SRC, int FMT>
+__device__ __forceinline__ uint8_t quant1_any(const void* src, int64_t e, const ScaleCtx& c) {
+    if constexpr (SRC == FP8DIT_SRC_BF16) {
+        return quant1<FMT>(static_cast<const uint16_t*>(src)[e], c);
+    } else {
+        float x;
+        uint32_t sign;
+        if constexpr (SRC == FP8DIT_SRC_F16) {
+            const uint16_t b = static_cast<const uint16_t*>(src)[e];
+            x = __half2float(__ushort_as_half(b));
+            sign = (b >> 8) & 0x80u;
+        } else {
+            x = static_cast<const float*>(src)[e];
+            sign = (__float_as_uint(x) >> 24) & 0x80u;
+        }
+        return (uint8_t)((codes2_div<FMT>(x, 0.0f, c.s) & 0xffu) | sign);
+    }
+}
+
+// Thread's share of the amax of chunk [begin, end) of a tensor, as |x| bits.
+template <int SRC>
+__device__ __forceinline__ uint32_t amax_chunk(const PerTensorDevDesc& d, int64_t begin, int64_t end) {
+    constexpr int EPV = Src<SRC>::kEpv;
+    constexpr int VPT = (int)(kChunk / EPV / kThreads);
+    const int64_t nvec = (end - begin) / EPV;  // whole vectors in this chunk
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(d.src) +
+                                                      begin * (SRC == FP8DIT_SRC_F32 ? 4 : 2));
+    uint32_t packed = 0;
+#pragma unroll 4
+    for (int i = 0; i < VPT; ++i) {
+        const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+        if (vi < nvec) packed = absmax_vec<SRC>(__ldg(src + vi), packed);
+    }
+    uint32_t m = SRC == FP8DIT_SRC_F32 ? packed : fold_halves(packed);
+    for (int64_t e = begin + nvec * EPV + threadIdx.x; e < end; e += kThreads) m = max(m, abs_bits1<SRC>(d.src, e));
+    return m;
+}
+
+// Codes of chunk [begin, end) of a tensor with scale context c.
+template <int SRC, int FMT>
+__device__ __forceinline__ void quant_chunk(const PerTensorDevDesc& d, int64_t begin, int64_t end, const ScaleCtx& c) {
+    constexpr int EPV = Src<SRC>::kEpv;
+    constexpr int VPT = (int)(kChunk / EPV / kThreads);
+    const int64_t nvec = (end - begin) / EPV;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(d.src) +
+                                                      begin * (SRC == FP8DIT_SRC_F32 ? 4 : 2));
+    uint8_t* dst = d.dst + begin;
+    if constexpr (SRC == FP8DIT_SRC_BF16) {
+        const Quot2 q2 = quot2_of(c);
+        if (c.fast) {
+#pragma unroll 4
+            for (int i = 0; i < VPT; ++i) {
+                const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+                if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT, true>(__ldcs(src + vi), q2));
+            }
+        } else {
+#pragma unroll 4
+            for (int i = 0; i < VPT; ++i) {
+                const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+                if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT, false>(__ldcs(src + vi), q2));
+            }
+        }
+    } else if constexpr (SRC == FP8DIT_SRC_F16) {
+#pragma unroll 4
+        for (int i = 0; i < VPT; ++i) {
+            const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+            if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant_vec_div<SRC, FMT>(__ldcs(src + vi), c.s));
+        }
+    } else {
+#pragma unroll 4
+        for (int i = 0; i < VPT; ++i) {
+            const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+            if (vi < nvec) __stcs(reinterpret_cast<uint32_t*>(dst) + vi, quant_vec_div<SRC, FMT>(__ldcs(src + vi), c.s).x);
+        }
+    }
+    for (int64_t e = begin + nvec * EPV + threadIdx.x; e < end; e += kThreads) d.dst[e] = quant1_any<SRC, FMT>(d.src, e, c);
 }
 
 template <int FMT>
@@ -73,24 +225,15 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
         const bool is_amax = off < amax_chunks_here;
         const int t = is_amax ? j : j - 1;
         const int64_t chunk = is_amax ? off : off - amax_chunks_here;
-        const PerTensorDevDesc d = a.d[t];
+        const PerTensorDevDesc& d = a.d[t];
         const int64_t begin = chunk * kChunk;
         const int64_t end = min(d.numel, begin + kChunk);
-        const int64_t nvec = (end - begin) >> 3;  // whole 8-element vectors in this chunk
-        const uint4* src = reinterpret_cast<const uint4*>(d.src + begin);
 
         if (is_amax) {
-            uint32_t packed = 0;
-#pragma unroll 4
-            for (int i = 0; i < kVecPerThread; ++i) {
-                const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
-                if (vi < nvec) {
-                    packed = absmax8(__ldg(src + vi), packed);
-                }
-            }
-            for (int64_t e = begin + nvec * 8 + threadIdx.x; e < end; e += kThreads)
-                packed = absmax2((uint32_t)d.src[e], packed);
-            uint32_t m = fold_halves(packed);
+            // The dtype is uniform across the block (one tensor per item).
+            uint32_t m = d.src_dtype == FP8DIT_SRC_F32   ? amax_chunk<FP8DIT_SRC_F32>(d, begin, end)
+                         : d.src_dtype == FP8DIT_SRC_F16 ? amax_chunk<FP8DIT_SRC_F16>(d, begin, end)
+                                                         : amax_chunk<FP8DIT_SRC_BF16>(d, begin, end);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
@@ -120,7 +263,10 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
                         }
                     }
                 }
-                const float amax = bf16_bits_to_float(ld_acquire_gpu(&a.amax_bits[t]));
+                const uint32_t bits = ld_acquire_gpu(&a.amax_bits[t]);
+                const float amax = d.src_dtype == FP8DIT_SRC_F32   ? abs_bits_to_float<FP8DIT_SRC_F32>(bits)
+                                   : d.src_dtype == FP8DIT_SRC_F16 ? abs_bits_to_float<FP8DIT_SRC_F16>(bits)
+                                                                   : abs_bits_to_float<FP8DIT_SRC_BF16>(bits);
                 s_amax = amax;
                 s_ok = ok;
                 if (ok && chunk == 0) *d.scale = scale_ctx<FMT>(amax).s;
@@ -128,23 +274,9 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
             __syncthreads();
             if (s_ok) {
                 const ScaleCtx c = scale_ctx<FMT>(s_amax);
-                const Quot2 q2 = quot2_of(c);
-                uint8_t* dst = d.dst + begin;
-                if (c.fast) {
-#pragma unroll 4
-                    for (int i = 0; i < kVecPerThread; ++i) {
-                        const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
-                        if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT, true>(__ldcs(src + vi), q2));
-                    }
-                } else {
-#pragma unroll 4
-                    for (int i = 0; i < kVecPerThread; ++i) {
-                        const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
-                        if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT, false>(__ldcs(src + vi), q2));
-                    }
-                }
-                for (int64_t e = begin + nvec * 8 + threadIdx.x; e < end; e += kThreads)
-                    d.dst[e] = quant1<FMT>(d.src[e], c);
+                if (d.src_dtype == FP8DIT_SRC_F32) quant_chunk<FP8DIT_SRC_F32, FMT>(d, begin, end, c);
+                else if (d.src_dtype == FP8DIT_SRC_F16) quant_chunk<FP8DIT_SRC_F16, FMT>(d, begin, end, c);
+                else quant_chunk<FP8DIT_SRC_BF16, FMT>(d, begin, end, c);
             }
         }
         __syncthreads();  // s_item / s_red / s_amax are rewritten next iteration
@@ -173,7 +305,7 @@ cudaError_t launch_per_tensor(const fp8dit_tensor_desc* host_descs, int32_t n, i
         int64_t total_chunks = 0;
         for (int32_t i = 0; i < nb; ++i) {
             const fp8dit_tensor_desc& h = host_descs[base + i];
-            args.d[i] = PerTensorDevDesc{h.src, h.numel, h.dst, h.scale};
+            args.d[i] = PerTensorDevDesc{h.src, h.numel, h.dst, h.scale, h.src_dtype};
             args.chunks[i] = (h.numel + kChunk - 1) / kChunk;
             total_chunks += args.chunks[i];
         }

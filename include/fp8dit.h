@@ -129,12 +129,21 @@ fp8dit_status fp8_quantize_weight_per_channel(const uint16_t* w, int64_t N, int6
                                               fp8dit_format fmt, uint8_t* qw, float* sw,
                                               fp8dit_stream_t stream);
 
+/* Element types a per-tensor conversion reads (a state-dict's floating dtypes). */
+typedef enum {
+    FP8DIT_SRC_BF16 = 0, /* bfloat16 bit patterns (the default: a zeroed field) */
+    FP8DIT_SRC_F16 = 1,  /* IEEE binary16 bit patterns */
+    FP8DIT_SRC_F32 = 2   /* IEEE binary32 */
+} fp8dit_src_dtype;
+
 /* One tensor of a per-tensor conversion. Pointers are device pointers. */
 typedef struct {
-    const uint16_t* src; /* numel bf16 values, contiguous, 16-byte aligned */
-    int64_t numel;       /* >= 0, any size */
-    uint8_t* dst;        /* numel FP8 codes, 16-byte aligned */
-    float* scale;        /* one fp32: S of the tensor (left untouched when numel == 0) */
+    const void* src;   /* numel values of src_dtype, contiguous, 16-byte aligned */
+    int64_t numel;     /* >= 0, any size */
+    uint8_t* dst;      /* numel FP8 codes, 16-byte aligned */
+    float* scale;      /* one fp32: S of the tensor (left untouched when numel == 0) */
+    int32_t src_dtype; /* fp8dit_src_dtype of src */
+    int32_t reserved;  /* must be 0 */
 } fp8dit_tensor_desc;
 
 /* Bytes of device workspace fp8_quantize_weight_per_tensor needs for n tensors. */
@@ -143,7 +152,10 @@ size_t fp8_quantize_weight_per_tensor_workspace_size(int32_t n_tensors);
 /*
  * Per-tensor conversion of a weight set (a state-dict's tensors) to FP8 with
  * one amax scale per tensor ("Quantize Model to FP8 Format": model_state_dict
- * in, quantised state-dict out in float8_e4m3fn or float8_e5m2).
+ * in, quantised state-dict out in float8_e4m3fn or float8_e5m2). Each tensor
+ * may be bf16, fp16 or fp32 (its src_dtype); every value is exact in fp32, so
+ * the recipe above applies unchanged: amax = max |x|, S = amax / fmax and
+ * q = RNEsat(x / S), both IEEE fp32 divisions.
  *   tensors   HOST array of n_tensors descriptors; it may be freed on return.
  *   workspace DEVICE scratch of at least
  *             fp8_quantize_weight_per_tensor_workspace_size(n_tensors) bytes,

@@ -7,7 +7,8 @@ never imports it and shares no code with it.
 What it computes (see oracle.c for the page citations):
   * ``decode`` / ``encode``: OCP E4M3FN and E5M2, round-half-even, saturating.
   * ``quantize_rows``: per-row amax, S = fp32(amax) / fmax, q = encode(x / S).
-  * ``quantize_tensor``: the same with one amax per tensor.
+  * ``quantize_tensor``: the same with one amax per tensor;
+    ``quantize_tensor_typed`` for bf16, fp16 or fp32 tensors.
   * ``linear``: exact integer dot of dequantised E4M3 operands, then
     y = dot * sa[m] * sw[n] + bias[n] in double.
   * ``linear_weight_only``: bf16 activation x decoded E4M3 weight, per-channel
@@ -61,6 +62,10 @@ def _load():
         lib.or_quantize_rows.argtypes = [_p, _i64, _i64, _i64, ctypes.c_int, _p, _i64, _p]
         lib.or_quantize_tensor.restype = None
         lib.or_quantize_tensor.argtypes = [_p, _i64, ctypes.c_int, _p, _p]
+        lib.or_quantize_tensor_typed.restype = None
+        lib.or_quantize_tensor_typed.argtypes = [_p, ctypes.c_int, _i64, ctypes.c_int, _p, _p]
+        lib.or_f16_to_f32.restype = ctypes.c_float
+        lib.or_f16_to_f32.argtypes = [ctypes.c_uint16]
         lib.or_linear.restype = None
         lib.or_linear.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _i64, _p]
         lib.or_linear_at.restype = None
@@ -121,6 +126,25 @@ def quantize_tensor(x: np.ndarray, fmt: int):
     s = np.empty((1,), dtype=np.float32)
     _load().or_quantize_tensor(x.ctypes.data, x.size, fmt, q.ctypes.data, s.ctypes.data)
     return q, float(s[0])
+
+
+SRC_BF16, SRC_F16, SRC_F32 = 0, 1, 2
+
+
+def quantize_tensor_typed(x: np.ndarray, fmt: int):
+    """Per-tensor quantisation of a bf16 (uint16 patterns), float16 or float32
+    array, any shape -> (q uint8 same shape, s float32 scalar)."""
+    src = {np.dtype(np.uint16): SRC_BF16, np.dtype(np.float16): SRC_F16, np.dtype(np.float32): SRC_F32}[x.dtype]
+    x = np.ascontiguousarray(x)
+    q = np.empty(x.shape, dtype=np.uint8)
+    s = np.empty((1,), dtype=np.float32)
+    _load().or_quantize_tensor_typed(x.ctypes.data, src, x.size, fmt, q.ctypes.data, s.ctypes.data)
+    return q, float(s[0])
+
+
+def f16_to_f32(bits: int) -> float:
+    """The oracle's closed-form decode of one binary16 bit pattern."""
+    return float(_load().or_f16_to_f32(bits))
 
 
 def linear(qa, sa, qw, sw, bias=None) -> np.ndarray:

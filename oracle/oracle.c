@@ -18,7 +18,8 @@
  *    run time) and section 三.1 (BF16 activation -> dynamic per-token FP8
  *    quant -> FP8 GEMM -> scale / bias / output dtype).
  *  - "Quantize Model to FP8 Format": whole state-dict tensors converted to
- *    float8_e4m3fn or float8_e5m2 with a scale (one scale per tensor).
+ *    float8_e4m3fn or float8_e5m2 with a scale (one scale per tensor); the
+ *    tensors may be bf16, fp16 or fp32.
  *
  * Formats (OCP 8-bit floating point, which the pages name):
  *  E4M3FN: bias 7, normal (-1)^s 2^(e-7) (1 + m/8), subnormal (-1)^s 2^-6 m/8,
@@ -145,6 +146,51 @@ void or_quantize_tensor(const uint16_t* x, int64_t n, int fmt, uint8_t* q, float
     *s = st;
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) q[i] = or_encode(fmt, or_bf16_to_f32(x[i]) / st);
+}
+
+/*
+ * fp16 bit pattern -> fp32, from the closed form of IEEE binary16: bias 15,
+ * normal (-1)^s 2^(e-15) (1 + m/1024), subnormal (-1)^s 2^-14 m/1024,
+ * exponent 31 is infinity (m = 0) or NaN. Every binary16 value is exact in fp32.
+ */
+float or_f16_to_f32(uint16_t h) {
+    int sign = h >> 15;
+    int e = (h >> 10) & 0x1F;
+    int m = h & 0x3FF;
+    double mag;
+    if (e == 31) mag = m == 0 ? INFINITY : NAN;
+    else if (e == 0) mag = ldexp((double)m / 1024.0, -14);
+    else mag = ldexp(1.0 + (double)m / 1024.0, e - 15);
+    return (float)(sign ? -mag : mag);
+}
+
+/* Element types a state-dict tensor may hold ("Quantize Model to FP8 Format":
+ * the node converts the model's floating weights, whatever their precision). */
+enum { OR_SRC_BF16 = 0, OR_SRC_F16 = 1, OR_SRC_F32 = 2 };
+
+static float load_elem(int src, const void* x, int64_t i) {
+    switch (src) {
+        case OR_SRC_F16:
+            return or_f16_to_f32(((const uint16_t*)x)[i]);
+        case OR_SRC_F32:
+            return ((const float*)x)[i];
+        default:
+            return or_bf16_to_f32(((const uint16_t*)x)[i]);
+    }
+}
+
+/* Per-tensor amax quantisation of n elements of type src (each exact in fp32):
+ * amax = max |x|, S = fp32(amax) / fmax, q = encode(x / S), as for bf16. */
+void or_quantize_tensor_typed(const void* x, int src, int64_t n, int fmt, uint8_t* q, float* s) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(load_elem(src, x, i));
+        if (a > amax) amax = a;
+    }
+    float st = scale_from_amax(fmt, amax);
+    *s = st;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) q[i] = or_encode(fmt, load_elem(src, x, i) / st);
 }
 
 /* ---------------------------------------------------------- linear */
