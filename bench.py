@@ -296,7 +296,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=("fp8dit", "reference"), default="fp8dit")
-    ap.add_argument("--no-extras", action="store_true", help="skip the attention / state-dict / bf16 extras")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the attention, state-dict and sustained measurements (and the context file)")
+    ap.add_argument("--extras-out", default=None,
+                    help="also measure the context figures (library GEMMs, variants, schedules) into this JSON file")
+    ap.add_argument("--sustained-s", type=float, default=2.0, help="seconds of back-to-back steps for `sustained`")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -346,6 +350,10 @@ def main():
     def gemm(name, i):
         b = sets[i % R][name]
         layers[name].forward_fp8(b["qa"], b["sa"], y=b["y"])
+
+    def linear(name, i):  # the whole layer from the bf16 activation: quantiser + GEMM
+        b = sets[i % R][name]
+        layers[name].forward(b["A"], y=b["y"], qa_scratch=b["qa"], sa_scratch=b["sa"])
 
     def step(i):
         for name, *_ in FFN:
@@ -404,72 +412,132 @@ def main():
     torch.cuda.synchronize()
     eager_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
 
-    # Per-kernel regions: each kernel alone, K back-to-back launches on the
-    # same rotating buffers (consecutive launches overlap launch and tail as
-    # in the step), captured in a CUDA graph and timed over one replay; the
-    # graph takes the host's per-call launch cost (~8 us from Python) out of
-    # the shorter kernels' figures.
+    # Per-kernel and per-layer regions: K back-to-back launches (or layer
+    # calls) on the rotating buffers, captured in a CUDA graph and timed over
+    # one replay; consecutive launches overlap launch and tail as in the step,
+    # and the graph takes the host's per-call launch cost (~8 us from Python)
+    # out of the shorter kernels' figures.
     k_avg = {}
     for name, *_ in FFN:
         k_avg[f"quantize_{name}"] = graph_region_ms(torch, lambda i, n=name: quantize(n, i), args.steps, dev, world)
         k_avg[f"gemm_{name}"] = graph_region_ms(torch, lambda i, n=name: gemm(n, i), args.steps, dev, world)
+    layer_ms = {name: graph_region_ms(torch, lambda i, n=name: linear(n, i), args.steps, dev, world)
+                for name, *_ in FFN}
     if fp8.device_error(dev) != 0:
         raise RuntimeError("device error during the per-kernel regions")
     step2_ms = sum(k_avg.values())
 
     value = whole_job_rate(world, FLOPS_PER_STEP, args.steps, elapsed_ms)
     peaks, peak_src = load_peaks()
-    region_s = elapsed_ms * 1e-3
-    sustained = region_s > 2.0
-    bf16_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    fp8_peak = bf16_peak * FP8_OVER_BF16
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16  # burst: every region above lasts milliseconds
+    fp8_peak_sustained = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
     hbm_peak = peaks["hbm_gbs"]
 
     gemm_us = (k_avg["gemm_up"] + k_avg["gemm_down"]) / 2 * 1e3
     gemm_flops = 2.0 * 4096 * 8192 * 2048
     gemm_tflops = gemm_flops / (gemm_us * 1e-6) / 1e12
     traffic = profiled_traffic("gemm_e4m3_kernel")
+    q_gbs = {n: QBYTES[n] / (k_avg[f"quantize_{n}"] * 1e-3) / 1e9 for n in ("up", "down")}
+    layer_tf = {n: 2.0 * M * N * K / (layer_ms[n] * 1e-3) / 1e12 for n, M, N, K in FFN}
     roofline = {"bound": "tensor", "kernel": "gemm_e4m3_kernel (FFN-up and FFN-down, mean)",
                 "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s", "frac": gemm_tflops / fp8_peak,
                 "traffic": traffic,
-                "timing": f"{args.steps} back-to-back launches per shape in one CUDA graph replay, "
-                          "CUDA events at the region ends",
-                "peak_source": f"{peak_src} bf16 {'sustained' if sustained else 'burst'} x {FP8_OVER_BF16:g} "
-                               f"(nominal FP8/BF16 ratio)"}
-    q_gbs = {n: QBYTES[n] / (k_avg[f"quantize_{n}"] * 1e-3) / 1e9 for n in ("up", "down")}
-    q_all = (QBYTES["up"] + QBYTES["down"]) / ((k_avg["quantize_up"] + k_avg["quantize_down"]) * 1e-3) / 1e9
-    quantizer = {"value": q_all, "unit": "GB/s", "frac_of_hbm": q_all / hbm_peak, "peak": hbm_peak,
-                 "ffn_up_gbs": q_gbs["up"], "ffn_down_gbs": q_gbs["down"],
-                 "bytes_per_step": QBYTES["up"] + QBYTES["down"]}
+                "peak_source": f"{peak_src} bf16 burst x {FP8_OVER_BF16:g} (nominal FP8/BF16 ratio)",
+                "linear_ffn_up_frac": layer_tf["up"] / fp8_peak, "linear_ffn_down_frac": layer_tf["down"] / fp8_peak,
+                "quantizer_ffn_up_frac": q_gbs["up"] / hbm_peak, "quantizer_ffn_down_frac": q_gbs["down"] / hbm_peak}
 
     # End to end through the public API with pinned host buffers.
     e2e = measure_e2e(fp8, torch, layers, host, dev, args, world)
+
+    targets = {}
+    for n, M, N, K in FFN:
+        targets[f"ffn_{n}"] = {
+            "linear_us": layer_ms[n] * 1e3, "linear_tflops": layer_tf[n], "linear_frac": layer_tf[n] / fp8_peak,
+            "quantize_us": k_avg[f"quantize_{n}"] * 1e3, "gemm_us": k_avg[f"gemm_{n}"] * 1e3,
+            "gemm_frac": 2.0 * M * N * K / (k_avg[f"gemm_{n}"] * 1e-3) / 1e12 / fp8_peak}
+    targets["quantizer"] = {"ffn_up_gbs": q_gbs["up"], "ffn_up_frac": q_gbs["up"] / hbm_peak,
+                            "ffn_down_gbs": q_gbs["down"], "ffn_down_frac": q_gbs["down"] / hbm_peak}
+    context = None
+    if world == 1 and rank == 0 and not args.no_extras:
+        att = measure_attention_and_state_dict(fp8, torch, synth, dev, up, fp8_peak, hbm_peak)
+        targets["quantizer"].update(att.pop("quantizer"))
+        targets.update(att)
+        targets["sustained"] = measure_sustained(torch, step, args, dev, fp8_peak_sustained)
+        if args.extras_out:
+            context = measure_context(fp8, torch, synth, dev, up, peaks, fp8_peak)
+    targets["peaks"] = {"fp8_tflops": fp8_peak, "fp8_tflops_sustained": fp8_peak_sustained, "hbm_gbs": hbm_peak,
+                        "source": peak_src}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 (bf16 in/out, fp32 accumulate)",
         "data": "synthetic", "config": config_dict(world),
-        "frac_of_fp8_peak": value / (fp8_peak * world),
-        "roofline": roofline, "quantizer": quantizer,
-        "kernels_us": {k: v * 1e3 for k, v in k_avg.items()},
-        "kernels_note": "per-kernel times: K back-to-back launches of each kernel alone, replayed from a "
-                        "CUDA graph (events at the ends); their sum "
-                        f"{step2_ms * 1e3:.1f} us vs the step's {elapsed_ms / args.steps * 1e3:.1f} us",
         "gpu_launches": 4 * args.steps,  # our kernels in timed region 1
         "timing": "K steps in one CUDA graph (captured after the W eager warm-up steps, replayed once untimed, "
                   "then once timed; events at the region ends)",
-        "eager_ms_per_step": eager_ms / args.steps,
-        "clocks": clk, "e2e": e2e,
+        "eager_ms_per_step": eager_ms / args.steps, "frac_of_fp8_peak": value / (fp8_peak * world),
+        "clocks": clk, "e2e": e2e, "roofline": roofline,
+        "kernels_us": {k: round(v * 1e3, 2) for k, v in k_avg.items()},
     }
-    if world == 1 and rank == 0 and not args.no_extras:
-        line["extras"] = measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
+        cb = cpu_baseline()
+        if context is not None:
+            context["cpu_baseline_components"] = cb.pop("components")
+        else:
+            cb.pop("components")
+        line["cpu_baseline"] = cb
+    line["targets"] = targets  # last: the end of the line carries every per-target figure
+    if context is not None:
+        context["kernels_note"] = (f"per-kernel times: K back-to-back launches of each kernel alone, replayed from a "
+                                   f"CUDA graph; their sum {step2_ms * 1e3:.1f} us vs the step's "
+                                   f"{elapsed_ms / args.steps * 1e3:.1f} us")
+        os.makedirs(os.path.dirname(os.path.abspath(args.extras_out)), exist_ok=True)
+        with open(args.extras_out, "w") as f:
+            json.dump(context, f, indent=1)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def measure_sustained(torch, step, args, dev, fp8_peak_sustained, n_steps=200):
+    """The step, back to back for at least --sustained-s seconds (a graph of
+    n_steps steps replayed repeatedly), with NVML clocks sampled meanwhile: the
+    regime a denoising loop runs in, against the sustained peak."""
+    cur = torch.cuda.current_stream(dev)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(cur)
+    with torch.cuda.stream(side):
+        step(0)
+    cur.wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        for i in range(n_steps):
+            step(i)
+    g.replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(cur)
+    g.replay()
+    b.record(cur)
+    torch.cuda.synchronize()
+    reps = max(1, int(args.sustained_s / max(a.elapsed_time(b) * 1e-3, 1e-6) + 0.5))
+    clocks = ClockSampler(dev, period_s=0.01)
+    clocks.start()
+    a.record(cur)
+    for _ in range(reps):
+        g.replay()
+    b.record(cur)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = a.elapsed_time(b)
+    del g
+    tf = FLOPS_PER_STEP * n_steps * reps / (ms * 1e-3) / 1e12
+    return {"seconds": ms * 1e-3, "steps": n_steps * reps, "tflops": tf, "frac": tf / fp8_peak_sustained,
+            "sm_mhz": clk["sm_mhz"], "reasons": clk["reasons"], "clock_samples": clk["samples"]}
 
 
 def measure_e2e(fp8, torch, layers, host, dev, args, world):
@@ -596,9 +664,13 @@ def scaled_mm_context(torch, layer, qs, ys, M, N, K, dev):
     return res
 
 
-def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
-    out = {}
-    # Attention projections: hidden [32760, 2048] quantised once, Q / K / V in one grouped launch.
+def measure_attention_and_state_dict(fp8, torch, synth, dev, up, fp8_peak, hbm_peak):
+    """The target figures beyond the FFN step: the rowwise quantiser on
+    hidden_states [32760, 2048]; the Q / K / V projections (one quantisation
+    feeding one grouped launch, HunyuanVideo page section 三.4) on
+    hidden_states and encoder_hidden_states, and the merged N = 6144
+    alternative; the per-tensor conversion of the 192-tensor weight set."""
+    out = {"quantizer": {}, "qkv": {}, "state_dict": {}}
     att = synth.attention()
     layers = [fp8.FP8Linear.from_weight(up(att[f"W_{p}"]), up(att[f"bias_{p}"])) for p in "qkv"]
     # The hidden_states quantiser alone, timed first: right after tens of ms of
@@ -609,8 +681,8 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
     sa = torch.empty((M,), dtype=torch.float32, device=dev)
     qms = graph_region_ms(torch, lambda i: fp8.quantize_rowwise(A[i % 2], q=qa, scale=sa), 50, dev)
     qb = 3 * M * 2048 + 4 * M
-    out["quantizer_hidden"] = {"us": qms * 1e3, "gbs": qb / (qms * 1e-3) / 1e9,
-                               "frac_of_hbm": qb / (qms * 1e-3) / 1e9 / hbm_peak}
+    out["quantizer"].update({"hidden_us": qms * 1e3, "hidden_gbs": qb / (qms * 1e-3) / 1e9,
+                             "hidden_frac": qb / (qms * 1e-3) / 1e9 / hbm_peak})
     # encoder_hidden_states first: its ~10 us launches are latency-bound and
     # read slower in the power state the hidden_states projections leave.
     for name in ("encoder", "hidden"):
@@ -622,8 +694,8 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
         ms = graph_region_ms(torch, lambda i: fp8.scaled_linear_multi(layers, A[i % 2], ys=ys[i % 2], qa_scratch=qa,
                                                                   sa_scratch=sa), 50, dev)
         flops = 3 * 2.0 * M * 2048 * 2048
-        out[f"attention_qkv_{name}"] = {"M": M, "us": ms * 1e3, "tflops": flops / (ms * 1e-3) / 1e12,
-                                        "frac_of_fp8_peak": flops / (ms * 1e-3) / 1e12 / fp8_peak}
+        out["qkv"][f"{name}_us"] = ms * 1e3
+        out["qkv"][f"{name}_frac"] = flops / (ms * 1e-3) / 1e12 / fp8_peak
     # Merged Q/K/V projection (one N = 6144 GEMM) vs the three separate,
     # grouped projections above, on hidden_states (HunyuanVideo page §三.4).
     A = [up(att["hidden"]) for _ in range(2)]
@@ -635,10 +707,30 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
     sa = torch.empty((M,), dtype=torch.float32, device=dev)
     ym = [torch.empty((M, 6144), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     ms = graph_region_ms(torch, lambda i: merged.forward(A[i % 2], y=ym[i % 2], qa_scratch=qa, sa_scratch=sa), 50, dev)
-    flops = 2.0 * M * 6144 * 2048
-    out["attention_qkv_merged_n6144"] = {"M": M, "us": ms * 1e3, "tflops": flops / (ms * 1e-3) / 1e12}
-    del A, ym
+    out["qkv"]["hidden_merged_n6144_us"] = ms * 1e3
+    del A, ym, merged, layers
+    # State-dict conversion: 192 tensors, 1.61e9 elements, both formats.
+    layout = synth.state_dict_layout()
+    tensors = [up(synth.state_dict_tensor(n, sh)) for n, sh in layout]
+    outs = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in tensors]
+    scales = torch.empty((len(tensors),), dtype=torch.float32, device=dev)
+    numel = sum(t.numel() for t in tensors)
+    alg_bytes = 3 * numel + 4 * len(tensors)
+    for fmt, fname in ((fp8.E4M3FN, "e4m3fn"), (fp8.E5M2, "e5m2")):
+        ms = time_region(torch, lambda i: fp8.quantize_per_tensor(tensors, fmt, outs=outs, scales=scales), 5, dev,
+                         warm=2)
+        out["state_dict"][f"{fname}_us"] = ms * 1e3
+        out["state_dict"][f"{fname}_gbs"] = alg_bytes / (ms * 1e-3) / 1e9
+        out["state_dict"][f"{fname}_frac"] = alg_bytes / (ms * 1e-3) / 1e9 / hbm_peak
+    del tensors, outs
+    return out
 
+
+def measure_context(fp8, torch, synth, dev, up, peaks, fp8_peak):
+    """Context figures, written to the --extras-out file: producer fusion,
+    GEMM-only times, the quantise-in-GEMM variant, the FP8 weight-only path,
+    BF16 and library FP8 GEMMs on the same shapes, stream-K and split-K."""
+    out = {}
     # Producer fusion (HunyuanVideo page §三.5): FFN-down fed by GELU(h), h the
     # FFN-up output. Fused: one kernel emits (FP8, scale). Unfused: torch's
     # bf16 GELU, then the rowwise quantiser. Both then run the FFN-down GEMM.
@@ -724,43 +816,29 @@ def measure_extras(fp8, torch, synth, dev, up, peaks, fp8_peak, hbm_peak):
                                       "stream_k_tflops": 2.0 * M * N * K / (sk_ms * 1e-3) / 1e12,
                                       "speedup": dp_ms / sk_ms}
     del qs, ys, layer
-    # Split-K against the plain schedule for text tokens through the FFN-down
-    # weight: [26, 8192] x [2048, 8192], 16 tiles of 128 x 128.
-    M = 26
-    layer = fp8.FP8Linear.from_weight(up(d["W"]), up(d["bias"]))
-    qs = [fp8.quantize_rowwise(up(synth.normal_bf16(f"bench/split/A{i}", (M, K), 1.0))) for i in range(3)]
-    ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(3)]
-    run = lambda i: layer.forward_fp8(qs[i % 3][0], qs[i % 3][1], y=ys[i % 3])
-    a16s = [up(synth.normal_bf16(f"bench/split/A16_{i}", (M, K), 1.0)) for i in range(3)]
-    run_wo = lambda i: layer.forward_weight_only(a16s[i % 3], y=ys[i % 3])
-    dp_ms = graph_region_ms(torch, run, 200, dev)
-    wo_ms = graph_region_ms(torch, run_wo, 200, dev)
-    layer.attach_workspace()
-    plan = list(layer.plan(M))
-    sp_ms = graph_region_ms(torch, run, 200, dev)
-    wos_ms = graph_region_ms(torch, run_wo, 200, dev)
-    layer.detach_workspace()
-    out["split_k_26x2048x8192"] = {"plain_us": dp_ms * 1e3, "split_k_us": sp_ms * 1e3, "split_plan": plan,
-                                   "speedup": dp_ms / sp_ms,
-                                   "w_gbs_split": N * K / (sp_ms * 1e-3) / 1e9,
-                                   "weight_only_plain_us": wo_ms * 1e3, "weight_only_split_k_us": wos_ms * 1e3,
-                                   "weight_only_speedup": wo_ms / wos_ms}
+    # Split-K against the plain schedule for few tokens through the FFN-down
+    # weight: [M, 8192] x [2048, 8192], 16 tiles of 128 x 128 (M = 26: the
+    # encoder_hidden_states length).
+    for M in (1, 26, 128):
+        layer = fp8.FP8Linear.from_weight(up(d["W"]), up(d["bias"]))
+        qs = [fp8.quantize_rowwise(up(synth.normal_bf16(f"bench/split/A{i}", (M, K), 1.0))) for i in range(3)]
+        ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        run = lambda i: layer.forward_fp8(qs[i % 3][0], qs[i % 3][1], y=ys[i % 3])
+        a16s = [up(synth.normal_bf16(f"bench/split/A16_{i}", (M, K), 1.0)) for i in range(3)]
+        run_wo = lambda i: layer.forward_weight_only(a16s[i % 3], y=ys[i % 3])
+        dp_ms = graph_region_ms(torch, run, 200, dev)
+        wo_ms = graph_region_ms(torch, run_wo, 200, dev)
+        layer.attach_workspace()
+        plan = list(layer.plan(M))
+        sp_ms = graph_region_ms(torch, run, 200, dev)
+        wos_ms = graph_region_ms(torch, run_wo, 200, dev)
+        layer.detach_workspace()
+        out[f"split_k_{M}x2048x8192"] = {"plain_us": dp_ms * 1e3, "split_k_us": sp_ms * 1e3, "split_plan": plan,
+                                         "speedup": dp_ms / sp_ms, "w_gbs_split": N * K / (sp_ms * 1e-3) / 1e9,
+                                         "weight_only_plain_us": wo_ms * 1e3,
+                                         "weight_only_split_k_us": wos_ms * 1e3,
+                                         "weight_only_speedup": wo_ms / wos_ms}
     del qs, ys, layer, a16s
-    # State-dict conversion: 192 tensors, 1.61e9 elements, both formats.
-    layout = synth.state_dict_layout()
-    tensors = []
-    for n, s in layout:
-        tensors.append(up(synth.state_dict_tensor(n, s)))
-    outs = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in tensors]
-    scales = torch.empty((len(tensors),), dtype=torch.float32, device=dev)
-    numel = sum(t.numel() for t in tensors)
-    alg_bytes = 3 * numel + 4 * len(tensors)
-    for fmt, fname in ((fp8.E4M3FN, "e4m3fn"), (fp8.E5M2, "e5m2")):
-        ms = time_region(torch, lambda i: fp8.quantize_per_tensor(tensors, fmt, outs=outs, scales=scales), 5, dev,
-                         warm=2)
-        out[f"state_dict_{fname}"] = {"tensors": len(tensors), "elements": numel, "us": ms * 1e3,
-                                      "gbs": alg_bytes / (ms * 1e-3) / 1e9,
-                                      "frac_of_hbm": alg_bytes / (ms * 1e-3) / 1e9 / hbm_peak}
     return out
 
 

@@ -288,10 +288,9 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
     const int64_t num_kb = (K + ke - 1) / ke;
     if (split > 1) {
         // One CTA per (tile, piece); tiles * split <= SMs by construction. The
-        // arrival counters and generation words (one each per tile, tiles <=
-        // SMs / 2) sit in the flag area after the stream-K flags, the partials
-        // in the partial area (tiles * split * 64 KB <= SMs * 64 KB, within
-        // (SMs / 2) * 256 KB).
+        // arrival counters (one per tile, tiles <= SMs / 2) sit in the flag
+        // area after the stream-K flags, the partials in the partial area
+        // (tiles * split * 64 KB <= SMs * 64 KB, within (SMs / 2) * 256 KB).
         const int pairs = hs[0]->num_sms / 2;
         units = tiles * split;
         if (units > dev->num_sms || (size_t)units * kSplitPieceBytes > (size_t)pairs * kSkPartialBytesPerUnit ||
@@ -299,7 +298,6 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
             return unsupported("split-K plan exceeds the workspace");
         args.split_k = split;
         args.split_arrive = static_cast<uint32_t*>(hs[0]->sk_ws) + split_flag_offset_words(pairs);
-        args.split_gen = args.split_arrive + pairs;
         args.sk_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(hs[0]->sk_ws) +
                                                    (stream_k_workspace_bytes(pairs) -
                                                     (size_t)pairs * kSkPartialBytesPerUnit));

@@ -110,10 +110,9 @@ struct alignas(64) GemmArgs {
     // Split-K (128 x 128 single-CTA tiles, few tiles): split_k > 1 pieces per
     // tile, CTA u computing piece u % split_k of tile u / split_k over an equal
     // share of the k-blocks. Every piece stores its fp32 partial and arrives on
-    // the tile's counter; the last arrival resets the counter and advances the
-    // tile's generation word, which the other pieces wait for; then each
-    // piece's CTA adds the split_k partials in piece order for its share of
-    // the tile's rows and writes y.
+    // the tile's counter; the arrival that completes the count resets it and
+    // its CTA adds the split_k partials in piece order for the whole tile and
+    // writes y. No piece waits for another.
     int32_t split_k;
     // Rows of A one TMA load brings per stage in the single-CTA FP8 plans:
     // M rounded up to 8 when M < 128 (one row tile), else 128. The MMA still
@@ -121,7 +120,6 @@ struct alignas(64) GemmArgs {
     // accumulator rows past M, which are never stored.
     int32_t a_box_rows;
     uint32_t* split_arrive;  // split-K: arrival counter per tile (zero between launches)
-    uint32_t* split_gen;     // split-K: generation word per tile (any value)
     uint32_t* sk_flag;   // stream-K: [units + 1][2 CTAs][8 epilogue warps] (zero between launches)
     float* sk_partial;   // stream-K: [units][2 CTAs][8 epilogue warps][32 rows][128 columns];
                          // split-K: [tiles][split_k][4 quarters][epilogue warps / 4 column parts]
@@ -131,8 +129,8 @@ struct alignas(64) GemmArgs {
 // Stream-K / split-K workspace for `units` CTA pairs: a flag area, then the
 // partials. The flag area holds the stream-K flags ((units + 1) x 16 words,
 // indexed by the unit that finishes a tile and its successor), then the
-// split-K arrival counters and generation words (units each: a split launch
-// has at most one tile per pair). Every region starts zeroed by
+// split-K arrival counters (one per tile: a split launch has at most one tile
+// per pair; followed by `units` spare words). Every region starts zeroed by
 // fp8_linear_set_workspace; stream-K flags and arrival counters return to
 // zero at the end of every launch, so one workspace serves any sequence of
 // stream-ordered launches of either schedule.
@@ -282,6 +280,21 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
             smem_u32(smem_dst)),
         "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+}
+
+// Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned) from global to this CTA's shared memory, completion counted on
+// `bar`. No multicast.
+__device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// Order global-memory accesses of the generic proxy (other threads' stores
+// this thread has acquired) before this thread's later async-proxy accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

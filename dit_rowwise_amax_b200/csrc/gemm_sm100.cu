@@ -42,8 +42,9 @@
 // workspace, stream-K (each unit an equal share of all k-blocks; a tile split
 // between two units is finished by one of them after the other has published
 // its fp32 partial) or split-K for few tiles and a long K (one CTA per (tile,
-// piece of K); once every piece has stored its fp32 partial, each adds the
-// pieces in order for its share of the rows), see SegSched.
+// piece of K); every piece stores its fp32 partial and arrives on the tile's
+// counter, and the piece that arrives last adds the pieces in order for the
+// whole tile), see SegSched.
 //
 // Every mbarrier wait is bounded (mbar_wait_bounded): on expiry the CTA
 // raises the device error word and its own and its peer's abort flags, lets
@@ -100,11 +101,14 @@ struct Cfg {
     static constexpr int STAGING_BYTES = EPI_WARPS * STG_BYTES;
     static constexpr int SWB_FLOATS = 2 * EPI_COLS;  // sw then bias as fp32, one copy per epilogue warp
     static constexpr int SWB_BYTES = EPI_WARPS * SWB_FLOATS * 4;
-    static constexpr int BAR_BYTES = 256;
+    static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_SMEM + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
     static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-    static_assert((3 * STAGES + 2 * ACC + 1) * 8 + 20 <= BAR_BYTES, "barrier area");
+    static_assert((3 * STAGES + 2 * ACC + 2) * 8 + 20 <= BAR_BYTES, "barrier area");
+    // Split-K reduction: one 32-row quarter of every piece's partial is staged
+    // in the (then idle) operand ring.
+    static_assert(!SPLIT_OK || kSplitMaxPieces * 32 * BN * 4 <= STAGES * STAGE_SMEM, "split-K staging");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(!W8 || (B_BYTES == 2 * RAW_BYTES && B_ROWS == 128), "in-place decode layout");
     static_assert(!AQ || ROWS == 128, "in-place quantise layout");
@@ -223,11 +227,12 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     uint64_t* tfull = conv + C::STAGES;
     uint64_t* tempty = tfull + C::ACC;
     uint64_t* drain = tempty + C::ACC;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* redbar = drain + 1;  // split-K: staged partial quarters landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redbar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile uint32_t* split_ticket = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);  // split-K
     volatile uint32_t* split_fail = reinterpret_cast<volatile uint32_t*>(tmem_slot + 3);    // split-K
-    volatile uint32_t* split_gen = reinterpret_cast<volatile uint32_t*>(tmem_slot + 4);     // split-K
+    volatile uint32_t* split_ok = reinterpret_cast<volatile uint32_t*>(tmem_slot + 4);      // split-K
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -252,10 +257,11 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             mbar_init(&tempty[a], C::EPI_WARPS * CG);  // one arrival per epilogue warp of the pair
         }
         mbar_init(drain, 1);
+        mbar_init(redbar, 1);
         *abort_flag = 0;
         *split_ticket = 0u;
         *split_fail = 0u;
-        *split_gen = 0u;
+        *split_ok = 0u;
         fence_mbarrier_init();
         tma_prefetch_desc(&args.tmA);
         for (int g = 0; g < args.G; ++g) {
@@ -458,62 +464,71 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             }
         };
 
-        // Split-K: once all pieces of tile t are stored, this CTA (piece p of
-        // S) adds, for rows [p R / S, (p + 1) R / S) of the tile's R valid
-        // rows, the S partials in piece order, applies the epilogue and stores
-        // bf16 to y. Thread i takes items i, i + 256, ...: item = (row, column
-        // float4 f), f fastest, so a warp's y stores are contiguous.
-        auto split_reduce = [&](int t, int p) {
+        // Split-K: the CTA whose arrival completes tile t's count adds, for
+        // every valid row of the tile, the S partials in piece order (the same
+        // order whichever piece arrives last, so results are deterministic),
+        // applies the epilogue and stores bf16 to y. The tile goes one 32-row
+        // quarter at a time: one thread bulk-copies that quarter of every
+        // piece's partial block ([quarter][column part][float4][row lane],
+        // 16 KB contiguous per piece) into the operand ring, which is idle by
+        // now (one segment per CTA), so the copy engine keeps the whole
+        // quarter in flight; then each thread sums float4 i of the S copies.
+        auto split_reduce = [&](int t) {
             const TileCoord tc = tile_coord(args, t);
             const GemmProblem& P = args.prob[tc.g];
             const int r0 = tc.tm * C::BM;
             const int rows = args.M - r0 < C::BM ? args.M - r0 : C::BM;
             const int c0 = tc.tn * BN;
-            const int cols = P.N - c0 < BN ? P.N - c0 : BN;
             const int S = args.split_k;
-            const int ra = (int)((int64_t)p * rows / S);
-            const int rb = (int)((int64_t)(p + 1) * rows / S);
-            constexpr int F4 = BN / 4;                        // float4 columns per row
-            constexpr size_t PIECE4 = (size_t)C::ROWS * BN / 4;  // float4 per piece
-            const float4* base = reinterpret_cast<const float4*>(args.sk_partial) + (size_t)t * S * PIECE4;
-            const int n_items = (rb - ra) * F4;
-            for (int i = ew * 32 + lane; i < n_items; i += 32 * C::EPI_WARPS) {
-                const int r = ra + i / F4;
-                const int f = i % F4;
-                if (4 * f >= cols) continue;
-                // Partial layout of a piece: [quarter q][column part h][float4 cv][row lane].
-                const int off = ((((r >> 5) * C::HALVES + f / (C::EPI_COLS / 4)) * (C::EPI_COLS / 4) +
-                                  f % (C::EPI_COLS / 4)) << 5) + (r & 31);
-                // Pieces in groups of four loads in flight, added in piece order.
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            constexpr uint32_t QBYTES = 32 * BN * 4;              // one quarter of one piece
+            constexpr int QF4 = (int)(QBYTES / 16);
+            constexpr size_t PIECE4 = (size_t)C::ROWS * BN / 4;   // float4 per piece
+            const float4* src = reinterpret_cast<const float4*>(args.sk_partial) + (size_t)t * S * PIECE4;
+            const float4* buf = reinterpret_cast<const float4*>(smem);
+            const int nq = (rows + 31) >> 5;
+            for (int qq = 0; qq < nq; ++qq) {
+                if (ew == 0 && lane == 0) {
+                    bool ok = *abort_flag == 0;
+                    if (ok) {
+                        if (qq == 0) fence_proxy_async_global();  // the acquired partials, before the copies
+                        mbar_arrive_expect_tx(redbar, (uint32_t)S * QBYTES);
+                        for (int p = 0; p < S; ++p)
+                            bulk_load_g2s(smem + (size_t)p * QBYTES, src + (size_t)p * PIECE4 + (size_t)qq * QF4,
+                                          QBYTES, redbar);
+                        ok = mbar_wait_bounded(redbar, (uint32_t)(qq & 1), abort_flag, args.err);
+                    }
+                    *split_ok = ok ? 1u : 0u;
+                }
+                named_barrier_sync(1, 32 * C::EPI_WARPS);
+                if (*split_ok != 1u) break;  // uniform: every epilogue thread reads the same word
+                for (int i = ew * 32 + lane; i < QF4; i += 32 * C::EPI_WARPS) {
+                    const int r = qq * 32 + (i & 31);
+                    const int f = i >> 5;  // float4 column of the tile
+                    const int n = c0 + 4 * f;
+                    if (r >= rows || n >= P.N) continue;
+                    float4 v = buf[i];
 #pragma unroll
-                for (int g = 0; g < kSplitMaxPieces; g += 4) {
-                    if (g >= S) break;
-                    float4 x[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        if (g + k < S) x[k] = __ldcg(base + (size_t)(g + k) * PIECE4 + off);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        if (g + k < S) {
-                            v.x += x[k].x;
-                            v.y += x[k].y;
-                            v.z += x[k].z;
-                            v.w += x[k].w;
+                    for (int p = 1; p < kSplitMaxPieces; ++p) {
+                        if (p < S) {
+                            const float4 x = buf[p * QF4 + i];
+                            v.x += x.x;
+                            v.y += x.y;
+                            v.z += x.z;
+                            v.w += x.w;
                         }
                     }
+                    const float sa = args.sa != nullptr ? __ldg(args.sa + r0 + r) : 1.0f;
+                    const float4 w4 = __ldg(reinterpret_cast<const float4*>(P.sw + n));
+                    uint2 b2 = make_uint2(0u, 0u);
+                    if (P.bias != nullptr) b2 = __ldg(reinterpret_cast<const uint2*>(P.bias + n));
+                    const float o0 = fmaf(v.x * sa, w4.x, __uint_as_float(b2.x << 16));
+                    const float o1 = fmaf(v.y * sa, w4.y, __uint_as_float(b2.x & 0xffff0000u));
+                    const float o2 = fmaf(v.z * sa, w4.z, __uint_as_float(b2.y << 16));
+                    const float o3 = fmaf(v.w * sa, w4.w, __uint_as_float(b2.y & 0xffff0000u));
+                    *reinterpret_cast<uint2*>(P.y + (size_t)(r0 + r) * P.N + n) =
+                        make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
                 }
-                const float sa = args.sa != nullptr ? __ldg(args.sa + r0 + r) : 1.0f;
-                const int n = c0 + 4 * f;
-                const float4 w4 = __ldg(reinterpret_cast<const float4*>(P.sw + n));
-                uint2 b2 = make_uint2(0u, 0u);
-                if (P.bias != nullptr) b2 = __ldg(reinterpret_cast<const uint2*>(P.bias + n));
-                const float o0 = fmaf(v.x * sa, w4.x, __uint_as_float(b2.x << 16));
-                const float o1 = fmaf(v.y * sa, w4.y, __uint_as_float(b2.x & 0xffff0000u));
-                const float o2 = fmaf(v.z * sa, w4.z, __uint_as_float(b2.y << 16));
-                const float o3 = fmaf(v.w * sa, w4.w, __uint_as_float(b2.y & 0xffff0000u));
-                *reinterpret_cast<uint2*>(P.y + (size_t)(r0 + r) * P.N + n) =
-                    make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+                named_barrier_sync(1, 32 * C::EPI_WARPS);  // every thread is done with the staged quarter
             }
         };
 
@@ -540,9 +555,6 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             // partial (32 rows x EPI_COLS fp32) is stored lane-fastest: float4 v
             // of row `lane` in column chunk c sits at [(c * 8 + v) * 32 + lane],
             // so every warp access moves 512 contiguous bytes.
-            // Split-K: the tile's generation before this piece arrives (read
-            // while the accumulator is still being built).
-            if (split && ew == 0 && lane == 0) *split_gen = ld_acquire_gpu_u32(args.split_gen + sg.t);
             const bool tail = !split && sg.k0 > 0;
             const bool head = !split && sg.k0 == 0 && sg.k1 < args.num_kb;
             const size_t part_elems = 32 * C::EPI_COLS;
@@ -697,44 +709,30 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 acc_phase ^= 1u;
             }
             if (split) {
-                // After all of this CTA's partial stores, thread 0 arrives on
-                // the tile's counter (acquire-release). The arrival that
-                // completes the count resets the counter and bumps the tile's
-                // generation word (release); every other piece waits, bounded,
-                // for the generation to move past the value it read before
-                // arriving. Then each piece reduces its share of the rows. The
-                // grid has one CTA per (tile, piece), at most one per SM, and
-                // each CTA allows the dependent launch only once it runs, so
-                // every piece is resident before any wait can matter. Every
-                // epilogue warp reaches every barrier on every path.
+                // Every thread fences its partial stores; after the barrier
+                // thread 0 arrives on the tile's counter (acquire-release).
+                // The arrival that completes the count sees every piece's
+                // partial, resets the counter for the next launch and reduces
+                // the whole tile; every other piece is done. No piece ever
+                // waits for another, so nothing depends on the pieces being
+                // resident at the same time (other kernels may hold SMs). A
+                // piece whose accumulator wait expired does not arrive: its
+                // tile stays unreduced and the device error word reports it.
                 uint32_t* arrive = args.split_arrive + sg.t;
-                uint32_t* gen = args.split_gen + sg.t;
                 if (failed && lane == 0) *split_fail = 1u;
+                __threadfence();
                 named_barrier_sync(1, 32 * C::EPI_WARPS);
                 if (ew == 0 && lane == 0) {
-                    bool ok = *split_fail == 0u;
-                    if (ok) {
-                        const uint32_t gen0 = *split_gen;
-                        if (atom_acq_rel_gpu_add_u32(arrive, 1u) == (uint32_t)args.split_k - 1u) {
-                            *arrive = 0u;
-                            st_release_gpu_u32(gen, gen0 + 1u);
-                        } else {
-                            const unsigned long long t0 = globaltimer_ns();
-                            while (ld_acquire_gpu_u32(gen) == gen0) {
-                                if (globaltimer_ns() - t0 > args.err.limit_ns) {
-                                    atomicOr(args.err.word, kDevErrTimeout);
-                                    ok = false;
-                                    break;
-                                }
-                                __nanosleep(32);
-                            }
-                        }
+                    uint32_t last = 0u;
+                    if (*split_fail == 0u && atom_acq_rel_gpu_add_u32(arrive, 1u) == (uint32_t)args.split_k - 1u) {
+                        *arrive = 0u;
+                        last = 1u;
                     }
-                    *split_ticket = ok ? 1u : 0u;
+                    *split_ticket = last;
                 }
                 named_barrier_sync(1, 32 * C::EPI_WARPS);
                 if (*split_ticket == 1u) {
-                    if constexpr (C::SPLIT_OK) split_reduce(sg.t, sg.piece);
+                    if constexpr (C::SPLIT_OK) split_reduce(sg.t);
                 }
             }
         }

@@ -194,13 +194,20 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  * an equal share of the layer's k-blocks; a tile split between two pairs is
  * finished by one of them after the other has stored its fp32 partial in this
  * workspace. Results stay deterministic (the two parts are added once, in
- * fp32) but differ in rounding from the plain schedule.
+ * fp32) but differ in rounding from the plain schedule. The finishing pair
+ * waits (bounded) for its partner's partial, which its partner computes
+ * first, so the schedule relies on all of the launch's pairs running at the
+ * same time: with other kernels holding SMs meanwhile, that wait may expire
+ * (FP8DIT_ERR_TIMEOUT).
  * The same workspace enables split-K for few tiles and a long K: when the
  * 128 x 128 tiles of a small-M call fill at most half of the SMs and K has at
  * least 48 k-blocks of 128 (K >= 6144; e.g. text tokens through an FFN-down
  * weight), each tile is cut into up to 8 pieces of at least 6 k-blocks on
- * separate CTAs; the pieces' fp32 partials are added in piece order
- * (deterministic, rounding differs from the plain schedule).
+ * separate CTAs; every piece stores its fp32 partial and the piece that
+ * arrives last adds all of them in piece order for the whole tile
+ * (deterministic, rounding differs from the plain schedule). No piece waits
+ * for another, so split-K launches need not have all their CTAs resident at
+ * once and may share the GPU with other kernels.
  * fp8_weight_only_linear splits the same way from 32 k-blocks of 64 (K >=
  * 2048; K >= 4096 above 64 rows). fp8_scaled_linear_multi uses the workspace
  * of its first layer. Without a workspace, or for other shapes (the
@@ -210,11 +217,11 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  *   fp8_linear_set_workspace: attach caller-owned DEVICE memory (256-byte
  *     aligned, at least that size) or detach with NULL, while no call that
  *     uses the layer is in flight. Attaching clears the workspace's flags
- *     (synchronously); every launch leaves them cleared (split-K's
- *     generation words excepted, which may hold any value), so
+ *     and counters (synchronously); every launch leaves them cleared, so
  *     stream-ordered launches and replays of a captured CUDA graph need no
  *     host reset. After a call whose device error word reports
- *     FP8DIT_ERR_TIMEOUT, attach the workspace again before reusing it. The
+ *     FP8DIT_ERR_TIMEOUT, attach the workspace again before reusing it (an
+ *     interrupted launch can leave a flag or a count behind). The
  *     workspace may be attached to several layers whose calls run one after
  *     another on the GPU; calls that overlap on the GPU must not share a
  *     workspace.

@@ -2,7 +2,9 @@
 the benchmark contract is present with a sensible value (metric and unit, the
 whole-job value, the timing fields, the roofline of the dominant kernel, the
 end-to-end figure with its host<->device bytes, the clocks sampled during the
-timed region, and the count of launches of the library's own kernels)."""
+timed region, the count of launches of the library's own kernels, and the
+per-target figures: each FFN linear from its bf16 activation and the
+quantiser per shape, against the measured peaks)."""
 import json
 import os
 import subprocess
@@ -45,3 +47,15 @@ def test_bench_json_line():
     for key in ("sm_mhz", "sm_max_mhz", "reasons"):
         assert key in c, key
     assert d["gpu_launches"] == 4 * d["steps"]  # two quantisers and two GEMMs per step
+    # The per-target figures sit in the last key, so the end of the line carries them.
+    assert list(d)[-1] == "targets"
+    t = d["targets"]
+    for layer in ("ffn_up", "ffn_down"):
+        for key in ("linear_us", "linear_tflops", "linear_frac", "quantize_us", "gemm_us", "gemm_frac"):
+            assert t[layer][key] > 0, (layer, key)
+        M, N, K = (4096, 8192, 2048) if layer == "ffn_up" else (4096, 2048, 8192)
+        assert t[layer]["linear_tflops"] == pytest.approx(2.0 * M * N * K / (t[layer]["linear_us"] * 1e-6) / 1e12)
+        assert t[layer]["linear_frac"] == pytest.approx(t[layer]["linear_tflops"] / t["peaks"]["fp8_tflops"])
+    for key in ("ffn_up_gbs", "ffn_up_frac", "ffn_down_gbs", "ffn_down_frac"):
+        assert t["quantizer"][key] > 0, key
+    assert rf["linear_ffn_up_frac"] == pytest.approx(t["ffn_up"]["linear_frac"])

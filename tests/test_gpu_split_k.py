@@ -1,11 +1,12 @@
 """Split-K schedule of the FP8 GEMM for few output tiles and a long K (small
 M, e.g. text tokens through an FFN-down weight). With a workspace attached,
 128 x 128 tiles filling at most half of the SMs and at least 48 k-blocks, each
-tile is cut into pieces along K on separate CTAs; once all pieces have stored
-their fp32 partials, each piece's CTA adds them in piece order for its share
-of the tile's rows and writes the output. Checked: the plan reports the split,
-every output against the oracle, the same bits on every run, no write outside
-y, graph replays, one workspace shared with stream-K, and the plain schedule
+tile is cut into pieces along K on separate CTAs; every piece stores its fp32
+partial and arrives on the tile's counter, and the piece that arrives last adds
+all of them in piece order and writes the tile. Checked: the plan reports the
+split, every output against the oracle, the same bits on every run, no write
+outside y, graph replays, one workspace shared with stream-K, concurrent
+launches on several streams, counters left cleared, and the plain schedule
 after detach and for a short K."""
 import numpy as np
 import pytest
@@ -228,31 +229,59 @@ def test_weight_only_split_k(M, N, K):
     assert torch.equal(y3.view(torch.int16), y_plain.view(torch.int16))
 
 
-TIMEOUT = 5  # FP8DIT_ERR_TIMEOUT
-
-
-def test_split_k_expired_wait_reports_timeout():
-    """A split-K arrival that can never complete: the first tile's arrival
-    counter is planted far above the piece count (the kind of state an
-    interrupted launch leaves), so no piece sees the count it waits for. Each
-    piece's bounded wait expires (about 2 s), the host reads
-    FP8DIT_ERR_TIMEOUT, and after the workspace is attached again (which
-    clears its counters) the same call gives the normal result."""
+def test_split_k_concurrent_launches_on_two_streams():
+    """Split-K launches of two layers (each with its own workspace) issued on
+    two streams so that they share the GPU, alongside a pair-tile GEMM on a
+    third stream. No piece waits for another (the last piece to arrive reduces
+    its tile), so nothing depends on all of a launch's CTAs being resident at
+    once: every launch completes, no device error is raised, and every output
+    equals the same call run alone, bit for bit."""
     M, N, K = 26, 2048, 8192
-    W = synth.normal_bf16(f"gpu/split/W/{N}x{K}", (N, K), 0.02)
-    layer, _, _ = layer_and_codes(W, synth.normal_bf16(f"gpu/split/b/{N}", (N,), 0.1))
+    layers, acts, refs = [], [], []
+    for i in range(2):
+        W = synth.normal_bf16(f"gpu/split/conc/W{i}", (N, K), 0.02)
+        layer, _, _ = layer_and_codes(W, synth.normal_bf16(f"gpu/split/conc/b{i}", (N,), 0.1))
+        layer.attach_workspace()
+        qa, sa = fp8.quantize_rowwise(to_device_bf16(synth.normal_bf16(f"gpu/split/conc/A{i}", (M, K), 1.0)))
+        layers.append(layer)
+        acts.append((qa, sa))
+        refs.append(layer.forward_fp8(qa, sa))
+    d = synth.ffn_up()
+    big = fp8.FP8Linear.from_weight(to_device_bf16(d["W"]), to_device_bf16(d["bias"]))
+    big_q = fp8.quantize_rowwise(to_device_bf16(d["A"]))
+    torch.cuda.synchronize()
+    assert fp8.device_error() == 0
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    outs = [[torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(20)] for _ in range(2)]
+    for it in range(20):
+        with torch.cuda.stream(streams[2]):
+            big.forward_fp8(*big_q)
+        for i in range(2):
+            with torch.cuda.stream(streams[i]):
+                layers[i].forward_fp8(*acts[i], y=outs[i][it])
+    torch.cuda.synchronize()
+    assert fp8.device_error() == 0
+    for i in range(2):
+        for it in range(20):
+            assert torch.equal(outs[i][it].view(torch.int16), refs[i].view(torch.int16)), (i, it)
+
+
+def test_split_k_leaves_counters_cleared():
+    """Every launch returns the workspace's flag area (stream-K flags and the
+    split-K arrival counters) to zero, so stream-ordered launches need no host
+    reset: after split-K launches of several shapes the area reads all zero."""
+    K = 8192
+    W = synth.normal_bf16(f"gpu/split/W/2048x{K}", (2048, K), 0.02)
+    layer, _, _ = layer_and_codes(W, synth.normal_bf16("gpu/split/b/2048", (2048,), 0.1))
     ws = layer.attach_workspace()
-    qa, sa = fp8.quantize_rowwise(to_device_bf16(synth.normal_bf16("gpu/split/timeout/A", (M, K), 1.0)))
-    y_ref = layer.forward_fp8(qa, sa)
+    for M in (1, 26, 128, 300):
+        qa, sa = fp8.quantize_rowwise(to_device_bf16(synth.normal_bf16(f"gpu/split/clr/A{M}", (M, K), 1.0)))
+        layer.forward_fp8(qa, sa)
+        layer.forward_weight_only(to_device_bf16(synth.normal_bf16(f"gpu/split/clr/A16{M}", (M, K), 1.0)))
+    torch.cuda.synchronize()
     assert fp8.device_error() == 0
     pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
-    arrive0 = (pairs + 1) * 16  # first split-K arrival counter, in 32-bit words (after the stream-K flags)
-    ws.view(torch.int32)[arrive0] = 1 << 30
-    torch.cuda.synchronize()
-    layer.forward_fp8(qa, sa)
-    assert fp8.device_error() == TIMEOUT
-    assert fp8.device_error() == 0  # reading clears the word
-    layer.attach_workspace(ws)  # clears the counters
-    y = layer.forward_fp8(qa, sa)
-    assert fp8.device_error() == 0
-    assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    partial_bytes = pairs * 2 * 8 * 32 * 128 * 4  # the fp32 partial area after the flags
+    flag_bytes = ws.numel() - partial_bytes
+    assert flag_bytes > 0
+    assert int(torch.count_nonzero(ws[:flag_bytes])) == 0
