@@ -291,6 +291,11 @@ __device__ __forceinline__ void bulk_load_g2s(void* smem_dst, const void* gsrc, 
                  "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
 }
+// Hint: bring `bytes` (a multiple of 16; address 16-byte aligned) of global
+// memory into L2. No data reaches the SM and nothing waits for it.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gsrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gsrc), "r"(bytes) : "memory");
+}
 // Order global-memory accesses of the generic proxy (other threads' stores
 // this thread has acquired) before this thread's later async-proxy accesses.
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -133,6 +133,19 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* _
 
     uint4 cur[VPT], nxt[VPT];
     int64_t g = blockIdx.x;
+    // Ask L2 for this block's first rows while the previous kernel in the
+    // stream is still finishing: a prefetch only warms L2, which every write
+    // of that kernel reaches too, so the loads after pdl_wait() still see its
+    // results. Each group is at most 256 threads x VPT x 16 bytes = 16 KB.
+    if (threadIdx.x == 0 && g < groups) {
+        const int64_t r0 = g * RPB;
+        const int64_t nr = M - r0 < RPB ? M - r0 : RPB;
+        if (ldx == K) {
+            prefetch_l2_bulk(x + r0 * ldx, (uint32_t)(nr * K * 2));
+        } else {
+            for (int64_t rr = 0; rr < nr; ++rr) prefetch_l2_bulk(x + (r0 + rr) * ldx, (uint32_t)K * 2u);
+        }
+    }
     pdl_wait();  // x may be the previous kernel's output; q and scale its input
     pdl_trigger();
     load_group<TPR, VPT>(x, M, nvec, ldx, g, cur);
