@@ -84,7 +84,7 @@ def load_library():
     L.fp8_scaled_linear_multi.argtypes = [ctypes.POINTER(p), i32, i64, p, p, p, ctypes.POINTER(p), p]
     L.fp8_scaled_linear_noalloc.argtypes = [p, i64, p, p, p]
     L.fp8_weight_only_linear.argtypes = [p, i64, p, p, p]
-    L.fp8_scaled_linear_fused.argtypes = [p, i64, p, p, p, p]
+    L.fp8_scaled_linear_fused.argtypes = [p, i64, p, p, p, p, p]
     L.fp8_linear_host_workspace_size.argtypes = [p, i64, i32]
     L.fp8_linear_host_workspace_size.restype = ctypes.c_size_t
     L.fp8_linear_set_host_pipeline.argtypes = [p, p, ctypes.c_size_t, i64, i32]
@@ -418,24 +418,33 @@ class FP8Linear:
         return y
 
     def forward_fused(self, a: torch.Tensor, y: Optional[torch.Tensor] = None,
-                      scale_scratch: Optional[torch.Tensor] = None) -> torch.Tensor:
-        """The FP8 linear from a bf16 activation with the per-token quantisation
-        done inside the GEMM (a row-scale pre-pass, then bf16 tiles quantised
-        to E4M3 in shared memory); same codes and result as forward().
-        scale_scratch: float32 [2 * M] (scales, then their reciprocals)."""
+                      qa_scratch: Optional[torch.Tensor] = None,
+                      sa_scratch: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """The FP8 linear from a bf16 activation in one launch: the launch's
+        CTAs quantise A per token (each element once) into qa_scratch /
+        sa_scratch, then run the GEMM, each tile starting once its rows are
+        quantised. Same codes, scales and (with 256 x 256 pair tiles) output
+        bits as forward(). Needs a workspace for its counters: one is attached
+        here if the layer has none (which also lets forward() use the stream-K
+        and split-K schedules)."""
         a = _bf16_matrix(a, "a")
         if not a.is_contiguous() or a.shape[1] != self.K:
             raise ValueError(f"a must be contiguous [M, {self.K}]")
         M = a.shape[0]
         _same_device(a, self.device, "a")
+        if getattr(self, "workspace", None) is None:
+            self.attach_workspace()
         if y is None:
             y = torch.empty((M, self.N), dtype=torch.bfloat16, device=a.device)
-        if scale_scratch is None:
-            scale_scratch = torch.empty((2 * M,), dtype=torch.float32, device=a.device)
+        if qa_scratch is None:
+            qa_scratch = torch.empty((M, self.K), dtype=torch.uint8, device=a.device)
+        if sa_scratch is None:
+            sa_scratch = torch.empty((M,), dtype=torch.float32, device=a.device)
         _check_out(y, "y", _BF16_DTYPES, (M, self.N), a.device)
-        _check_out(scale_scratch, "scale_scratch", (torch.float32,), (2 * M,), a.device)
-        _check(load_library().fp8_scaled_linear_fused(self._h, M, a.data_ptr(), scale_scratch.data_ptr(),
-                                                      y.data_ptr(), _stream(a.device)))
+        _check_out(qa_scratch, "qa_scratch", _CODE_DTYPES, (M, self.K), a.device)
+        _check_out(sa_scratch, "sa_scratch", (torch.float32,), (M,), a.device)
+        _check(load_library().fp8_scaled_linear_fused(self._h, M, a.data_ptr(), qa_scratch.data_ptr(),
+                                                      sa_scratch.data_ptr(), y.data_ptr(), _stream(a.device)))
         return y
 
     def attach_host_pipeline(self, chunk_rows: int = 2048, slots: int = 2) -> torch.Tensor:

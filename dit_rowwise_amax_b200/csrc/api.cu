@@ -186,12 +186,19 @@ static int choose_cfg_weight_only(const fp8dit_linear_s* h, int64_t M) {
     return kCfgW8128x128;
 }
 
-// Quantise-in-GEMM plan: the same choice between pair tiles and 128 x 128 tiles.
+// Fused-linear plan: the same choice between pair tiles and 128 x 128 tiles.
 static int choose_cfg_fused(const fp8dit_linear_s* h, int64_t M) {
     const int pairs = h->num_sms / 2;
-    if (M >= 256 && tiles_for(h, M, 1, kCfgAQPair256) * 2 >= pairs) return kCfgAQPair256;
-    return kCfgAQ128x128;
+    if (M >= 256 && tiles_for(h, M, 1, kCfgQGPair256) * 2 >= pairs) return kCfgQGPair256;
+    return kCfgQG128x128;
 }
+
+// What the fused linear's launch needs besides the GEMM's operands.
+struct QgInputs {
+    const uint16_t* a;  // bf16 A [M, K]
+    uint8_t* qa;        // its codes (the GEMM's A)
+    float* sa;          // its scales
+};
 
 // Split-K plan for the single-CTA plans of the FP8 linear and of the
 // weight-only linear when a workspace is attached: if 128 x 128 tiles fill at
@@ -228,12 +235,13 @@ static int a_box_rows_for(int cfg, int64_t M) {
     return (gemm_cta_group(cfg) == 1 && M < 128) ? (int)((M + 7) / 8 * 8) : 128;
 }
 
-// a: FP8 codes [M, K] (qa) for the FP8 x FP8 configurations, bf16 [M, K] for
-// the weight-only and quantise-in-GEMM ones; sa: per-token scales, or NULL
-// (weight-only); ra: the per-token reciprocals (quantise-in-GEMM only).
+// a: FP8 codes [M, K] (qa) for the FP8 x FP8 configurations (the fused
+// linear's included: the launch writes them first), bf16 [M, K] for the
+// weight-only ones; sa: per-token scales, or NULL (weight-only); qg: the
+// fused linear's bf16 activation and outputs.
 static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, const void* a, const float* sa,
                               uint16_t* const* ys, cudaStream_t stream, const DeviceInfo* dev, int cfg,
-                              const float* ra = nullptr) {
+                              const QgInputs* qg = nullptr) {
     const int split = split_pieces(hs, n, M, cfg, dev->num_sms);
     if (split > 1 && !gemm_weight_only(cfg)) cfg = kCfg128x128;
     const int bm = gemm_block_m(cfg);
@@ -243,15 +251,11 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
     GemmArgs args;
     memset(&args, 0, sizeof(args));
     // A: FP8 codes (128-byte rows, swizzled, MMA-ready); weight-only: bf16
-    // (128-byte rows of 64 elements, swizzled, MMA-ready); quantise-in-GEMM:
-    // bf16 rows of 128 elements (256 bytes, unswizzled), quantised in shared memory.
+    // (128-byte rows of 64 elements, swizzled, MMA-ready).
     fp8dit_status st =
         gemm_weight_only(cfg)
             ? encode_tma_2d(&args.tmA, 2, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, (uint32_t)ke, 128,
                             CU_TENSOR_MAP_SWIZZLE_128B)
-        : gemm_quantizes_a(cfg)
-            ? encode_tma_2d(&args.tmA, 2, a, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, (uint32_t)ke, 128,
-                            CU_TENSOR_MAP_SWIZZLE_NONE)
             : encode_tma_2d(&args.tmA, 1, a, (uint64_t)K, (uint64_t)M, (uint64_t)K, (uint32_t)ke,
                             (uint32_t)a_box_rows_for(cfg, M), CU_TENSOR_MAP_SWIZZLE_128B);
     args.a_box_rows = a_box_rows_for(cfg, M);
@@ -313,7 +317,22 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
         }
     }
     args.sa = sa;
-    args.ra = ra;
+    if (qg != nullptr) {
+        // Rows per staged chunk: a power of two dividing 128 whose bf16 rows
+        // fit one staging buffer; threads per row: the smallest power of two
+        // (8 .. 256) that covers a row with at most four 16-byte vectors each.
+        int rows = 128;
+        while (rows > 1 && (uint64_t)rows * (uint64_t)K * 2 > kQgBufBytes) rows >>= 1;
+        int tpr = 8;
+        while (tpr * 4 < K / 8) tpr *= 2;
+        args.qg_a = qg->a;
+        args.qg_q = qg->qa;
+        args.qg_s = qg->sa;
+        args.qg_ctr = static_cast<uint32_t*>(hs[0]->sk_ws) + qg_offset_words(hs[0]->num_sms / 2);
+        args.qg_rows = rows;
+        args.qg_tpr = tpr;
+        args.qg_chunks = (int32_t)((M + rows - 1) / rows);
+    }
     args.M = (int32_t)M;
     args.K = (int32_t)hs[0]->K;
     args.G = n;
@@ -564,26 +583,25 @@ fp8dit_status fp8_weight_only_linear(fp8dit_linear h, int64_t M, const uint16_t*
     return run_gemm(&h, 1, M, a_bf16, nullptr, &y, (cudaStream_t)stream, dev, choose_cfg_weight_only(h, M));
 }
 
-fp8dit_status fp8_scaled_linear_fused(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, float* scale_scratch,
-                                      uint16_t* y, fp8dit_stream_t stream) {
+fp8dit_status fp8_scaled_linear_fused(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, uint8_t* qa_scratch,
+                                      float* sa_scratch, uint16_t* y, fp8dit_stream_t stream) {
     t_last_error[0] = 0;
     if (!h) return invalid("null handle");
     if (M < 0) return invalid("M must be >= 0");
-    if (M > kMaxRows) return unsupported("M too large");
+    if (M > (int64_t)kQgMaxRowBlocks * 128) return unsupported("the fused linear takes at most 1048576 rows");
+    if (h->K > kQgMaxK) return unsupported("the fused linear takes K <= 8192");
     if (M == 0) return FP8DIT_OK;
     if (!a_bf16 || !aligned16(a_bf16)) return invalid("a_bf16 must be non-null and 16-byte aligned");
-    if (!scale_scratch || ((uintptr_t)scale_scratch & 3u) != 0)
-        return invalid("scale_scratch must be non-null and 4-byte aligned");
+    if (!qa_scratch || !aligned16(qa_scratch)) return invalid("qa_scratch must be non-null and 16-byte aligned");
+    if (!sa_scratch || ((uintptr_t)sa_scratch & 3u) != 0) return invalid("sa_scratch must be non-null and 4-byte aligned");
     if (!y || !aligned16(y)) return invalid("y must be non-null and 16-byte aligned");
+    if (h->sk_ws == nullptr) return invalid("the fused linear needs a workspace (fp8_linear_set_workspace)");
     fp8dit_status st = check_device(h);
     if (st != FP8DIT_OK) return st;
     const DeviceInfo* dev = device_info();
     if (!dev) return FP8DIT_ERR_CUDA;
-    float* sa = scale_scratch;
-    float* ra = scale_scratch + M;
-    cudaError_t e = launch_row_scales(a_bf16, M, h->K, h->K, sa, ra, (cudaStream_t)stream, dev);
-    if (e != cudaSuccess) return cuda_fail(e, "row scale launch");
-    return run_gemm(&h, 1, M, a_bf16, sa, &y, (cudaStream_t)stream, dev, choose_cfg_fused(h, M), ra);
+    const QgInputs qg{a_bf16, qa_scratch, sa_scratch};
+    return run_gemm(&h, 1, M, qa_scratch, sa_scratch, &y, (cudaStream_t)stream, dev, choose_cfg_fused(h, M), &qg);
 }
 
 fp8dit_status fp8_scaled_linear_multi(const fp8dit_linear* hs, int32_t n, int64_t M, const uint16_t* a_bf16,

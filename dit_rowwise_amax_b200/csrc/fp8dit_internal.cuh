@@ -54,11 +54,6 @@ fp8dit_status encode_tma_2d(CUtensorMap* map, int elem_bytes, const void* base, 
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int fmt,
                                  uint8_t* q, int64_t ldq, float* scale, cudaStream_t stream,
                                  const DeviceInfo* dev);
-// Per-row E4M3 scales S = amax / 448 (1 for an all-zero row) and, where the
-// corrected-reciprocal quotient applies, rcp = RN(1 / S) (else 0): what the
-// rowwise quantiser uses, without writing codes.
-cudaError_t launch_row_scales(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float* scale, float* rcp,
-                              cudaStream_t stream, const DeviceInfo* dev);
 cudaError_t launch_act_quantize_rows(const uint16_t* h, int64_t M, int64_t K, int64_t ldh, int act, uint8_t* q,
                                      int64_t ldq, float* scale, uint16_t* g, int64_t ldg, cudaStream_t stream,
                                      const DeviceInfo* dev);
@@ -95,7 +90,6 @@ struct alignas(64) GemmArgs {
     CUtensorMap tmY[kMaxGroups];   // y bf16 [M, N], box 32 x 32, 64-byte swizzle (TMA store)
     GemmProblem prob[kMaxGroups];
     const float* sa;
-    const float* ra;  // AQ: RN(1 / sa[m]) where the corrected-reciprocal quotient applies, else 0
     int32_t M, K, G;
     int32_t tiles_m;
     int32_t num_tiles;
@@ -120,6 +114,15 @@ struct alignas(64) GemmArgs {
     // accumulator rows past M, which are never stored.
     int32_t a_box_rows;
     uint32_t* split_arrive;  // split-K: arrival counter per tile (zero between launches)
+    // Fused linear (quantise, then GEMM, in one launch): bf16 A, written into
+    // the FP8 A that tmA describes and the scales sa by the launch itself.
+    const uint16_t* qg_a;  // bf16 A [M, K], contiguous
+    uint8_t* qg_q;         // its E4M3 codes [M, K] (what tmA describes)
+    float* qg_s;           // its per-token scales [M] (== sa)
+    uint32_t* qg_ctr;      // [0] chunks claimed, [1] CTAs finished, [2 + b] rows of 128-row block b quantised
+    int32_t qg_rows;       // rows per chunk (a power of two dividing 128; rows x K x 2 <= kQgBufBytes)
+    int32_t qg_tpr;        // threads per row (power of two, 8..256) in the quantising warps
+    int32_t qg_chunks;     // ceil(M / qg_rows)
     uint32_t* sk_flag;   // stream-K: [units + 1][2 CTAs][8 epilogue warps] (zero between launches)
     float* sk_partial;   // stream-K: [units][2 CTAs][8 epilogue warps][32 rows][128 columns];
                          // split-K: [tiles][split_k][4 quarters][epilogue warps / 4 column parts]
@@ -130,13 +133,22 @@ struct alignas(64) GemmArgs {
 // partials. The flag area holds the stream-K flags ((units + 1) x 16 words,
 // indexed by the unit that finishes a tile and its successor), then the
 // split-K arrival counters (one per tile: a split launch has at most one tile
-// per pair; followed by `units` spare words). Every region starts zeroed by
-// fp8_linear_set_workspace; stream-K flags and arrival counters return to
-// zero at the end of every launch, so one workspace serves any sequence of
-// stream-ordered launches of either schedule.
+// per pair; followed by `units` spare words), then the fused linear's
+// counters (2 + kQgMaxRowBlocks words). Every region starts zeroed by
+// fp8_linear_set_workspace; stream-K flags and all counters return to zero at
+// the end of every launch, so one workspace serves any sequence of
+// stream-ordered launches of any schedule.
 constexpr size_t kSkFlagBytesPerUnit = 2 * 8 * sizeof(uint32_t);
 inline size_t sk_flag_words(int units) { return (size_t)(units + 1) * 16; }
 inline size_t split_flag_offset_words(int units) { return sk_flag_words(units); }
+// Fused linear: rows are quantised in chunks staged in shared memory, at most
+// kQgBufs chunks of kQgBufBytes in flight per CTA; readiness is counted per
+// 128-row block, so M <= 128 x kQgMaxRowBlocks; rows up to kQgMaxK elements.
+constexpr int kQgBufs = 3;
+constexpr uint32_t kQgBufBytes = 65536;
+constexpr int kQgMaxRowBlocks = 8192;
+constexpr int kQgMaxK = 8192;
+inline size_t qg_offset_words(int units) { return split_flag_offset_words(units) + 2 * (size_t)units; }
 constexpr size_t kSkPartialBytesPerUnit = 2 * 8 * 32 * 128 * sizeof(float);
 constexpr int64_t kSkMinKBlocks = 8;  // shorter tiles gain less from a split than it costs
 // Split-K pays where a single-CTA tile's k-loop, which at small M is bound by
@@ -150,7 +162,7 @@ constexpr int kSplitMinKBlocks = 6;        // split-K: k-blocks per piece (one r
 constexpr int kSplitMaxPieces = 8;         // split-K: pieces per tile, at most
 constexpr size_t kSplitPieceBytes = 128 * 128 * sizeof(float);  // one fp32 128 x 128 partial
 inline size_t stream_k_workspace_bytes(int units) {
-    const size_t flags = ((sk_flag_words(units) + 2 * (size_t)units) * sizeof(uint32_t) + 4095) & ~(size_t)4095;
+    const size_t flags = ((qg_offset_words(units) + 2 + kQgMaxRowBlocks) * sizeof(uint32_t) + 4095) & ~(size_t)4095;
     return flags + (size_t)units * kSkPartialBytesPerUnit;
 }
 
@@ -161,8 +173,8 @@ enum GemmConfig : int32_t {
     kCfg128x128 = 2,    // FP8 x FP8: 128 x 128 tile on one CTA
     kCfgW8Pair256 = 3,  // bf16 x FP8 weight (weight-only): 256 x 256 tile on a 2-CTA pair
     kCfgW8128x128 = 4,  // bf16 x FP8 weight (weight-only): 128 x 128 tile on one CTA
-    kCfgAQPair256 = 5,  // bf16 A quantised in the GEMM x FP8 weight: 256 x 256 tile on a 2-CTA pair
-    kCfgAQ128x128 = 6,  // bf16 A quantised in the GEMM x FP8 weight: 128 x 128 tile on one CTA
+    kCfgQGPair256 = 5,  // fused linear (bf16 A quantised by the launch, then FP8 x FP8): 256 x 256 pair tile
+    kCfgQG128x128 = 6,  // fused linear: 128 x 128 tile on one CTA
     kCfg128x64 = 7,     // FP8 x FP8: 128 x 64 tile on one CTA (few rows: deeper ring, more CTAs)
     kNumCfgs = 8,
 };
@@ -171,7 +183,7 @@ int gemm_block_n(int cfg);
 int gemm_b_box_rows(int cfg);
 int gemm_cta_group(int cfg);
 bool gemm_weight_only(int cfg);
-bool gemm_quantizes_a(int cfg);  // bf16 A quantised in the kernel (per-row scales sa, reciprocals ra)
+bool gemm_quantizes_a(int cfg);  // fused linear: bf16 A quantised by the launch before its GEMM
 int gemm_k_elems(int cfg);  // K elements per pipeline stage
 constexpr int kGemmBlockK = 128;  // bytes = FP8 elements per k-block (one 128 B swizzle row)
 constexpr int kGemmStoreBox = 32;

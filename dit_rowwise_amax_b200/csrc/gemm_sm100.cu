@@ -33,10 +33,11 @@
 //
 // Operand modes (OPS): kOpsFp8 is the FP8 linear above. kOpsW8 (FP8
 // weight-only: bf16 A x E4M3 W, "longcat-avatar-compare", section 速度总览)
-// and kOpsAQ (bf16 A quantised per token inside the GEMM) add one converter
-// warp per ring stage after the epilogue warps, which turns the stage's W codes
-// into bf16 (W8) or its bf16 A tile into E4M3 codes (AQ) in place in shared
-// memory before releasing the stage to the MMA.
+// adds one converter warp per ring stage after the epilogue warps, which turns
+// the stage's W codes into bf16 in place in shared memory before releasing the
+// stage to the MMA. kOpsQG (the fused linear) first quantises the bf16 A per
+// token with every CTA of the launch (phase Q, see qg_quantise), then runs the
+// kOpsFp8 GEMM on the codes.
 //
 // Schedules: data-parallel (tile t on MMA unit t mod units) or, with a
 // workspace, stream-K (each unit an equal share of all k-blocks; a tile split
@@ -62,31 +63,31 @@ namespace {
 // Operand modes of the kernel.
 //   kOpsFp8: A and W are FP8 codes, both loaded by TMA (the FP8 linear).
 //   kOpsW8:  A is bf16; W codes are decoded to bf16 in shared memory (weight-only).
-//   kOpsAQ:  A is bf16 and is quantised to FP8 in shared memory with per-row
-//            scales computed beforehand; W is FP8 (quantise-in-GEMM variant).
-enum : int { kOpsFp8 = 0, kOpsW8 = 1, kOpsAQ = 2 };
+//   kOpsQG:  A is bf16: the launch's CTAs first quantise it per token into the
+//            caller's FP8 scratch (rows claimed chunk by chunk, staged in
+//            shared memory), then run the kOpsFp8 GEMM on it, each tile
+//            starting once its rows are quantised (the fused linear).
+enum : int { kOpsFp8 = 0, kOpsW8 = 1, kOpsQG = 2 };
 
 template <int CG, int BN, int OPS>
 struct Cfg {
     static constexpr bool W8 = OPS == kOpsW8;
-    static constexpr bool AQ = OPS == kOpsAQ;
-    static constexpr bool CONV = W8 || AQ;  // has converter warps
+    static constexpr bool QG = OPS == kOpsQG;
+    static constexpr bool CONV = W8;        // has converter warps
     static constexpr int BM = 128 * CG;     // rows of one MMA tile
     static constexpr int ROWS = 128;        // rows per CTA (TMEM lanes)
     static constexpr int ROW_BYTES = 128;   // one 128-byte swizzle row per operand row per stage
     static constexpr int KE = W8 ? 64 : 128;  // K elements per stage (bf16 : FP8)
     static constexpr int B_ROWS = BN / CG;  // W rows per CTA per stage
     static constexpr int A_BYTES = ROWS * ROW_BYTES;  // MMA-ready A per stage
-    // AQ: the bf16 A tile as loaded (ROWS rows x 256 bytes) fills the stage's
-    // A buffer and is quantised in place into its first A_BYTES.
-    static constexpr int A_STAGE = AQ ? 2 * A_BYTES : A_BYTES;
+    static constexpr int A_STAGE = A_BYTES;
     static constexpr int B_BYTES = B_ROWS * ROW_BYTES;         // MMA-ready B: FP8, or bf16 decoded from FP8
     // W8: the FP8 weight codes as loaded (B_ROWS rows x 64 bytes) land in the
     // upper half of the stage's B buffer and are decoded in place.
     static constexpr int RAW_BYTES = W8 ? B_ROWS * 64 : 0;
     static constexpr int TX_BYTES = A_STAGE + (W8 ? RAW_BYTES : B_BYTES);  // TMA bytes per CTA per stage
     static constexpr int STAGE_SMEM = A_STAGE + B_BYTES;
-    static constexpr int STAGES = W8 ? 6 : AQ ? 4 : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : BN == 64 ? 8 : 6));
+    static constexpr int STAGES = W8 ? 6 : ((CG == 2) ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : BN == 64 ? 8 : 6));
     static constexpr int ACC = 2;
     static constexpr uint32_t TMEM_COLS = ACC * BN;
     static constexpr int EPI_WARPS = CONV ? 4 : 8;   // one or two per TMEM lane quarter
@@ -105,13 +106,15 @@ struct Cfg {
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_SMEM + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
     static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-    static_assert((3 * STAGES + 2 * ACC + 2) * 8 + 20 <= BAR_BYTES, "barrier area");
+    static_assert((3 * STAGES + 2 * ACC + 2 + 2 * kQgBufs) * 8 + 4 * 32 <= BAR_BYTES, "barrier area");
+    // Fused linear: kQgBufs chunks of bf16 rows (kQgBufBytes each) are staged
+    // in the operand ring before the GEMM uses it.
+    static_assert(!QG || kQgBufs * kQgBufBytes <= STAGES * STAGE_SMEM, "quantiser staging");
     // Split-K reduction: one 32-row quarter of every piece's partial is staged
     // in the (then idle) operand ring.
     static_assert(!SPLIT_OK || kSplitMaxPieces * 32 * BN * 4 <= STAGES * STAGE_SMEM, "split-K staging");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(!W8 || (B_BYTES == 2 * RAW_BYTES && B_ROWS == 128), "in-place decode layout");
-    static_assert(!AQ || ROWS == 128, "in-place quantise layout");
 };
 
 struct TileCoord {
@@ -199,6 +202,26 @@ __device__ __forceinline__ uint32_t atom_acq_rel_gpu_add_u32(uint32_t* p, uint32
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
 }
+// Wait (acquire, bounded) until *p == want. Gives up when *abort becomes
+// non-zero or after err.limit_ns (then raises *abort and the error word).
+__device__ __forceinline__ bool wait_count_bounded(const uint32_t* p, uint32_t want, volatile int* abort,
+                                                   const DevErr& err) {
+    if (ld_acquire_gpu_u32(p) == want) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire_gpu_u32(p) == want) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > err.limit_ns) {
+            *abort = 1;
+            atomicOr(err.word, kDevErrTimeout);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void red_add_release_gpu_u32(uint32_t* p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ void st_release_gpu_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -213,7 +236,6 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     gemm_e4m3_kernel(const __grid_constant__ GemmArgs args) {
     using C = Cfg<CG, BN, OPS>;
     constexpr bool W8 = C::W8;
-    constexpr bool AQ = C::AQ;
     constexpr bool CONV = C::CONV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -223,16 +245,22 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     float* swb = reinterpret_cast<float*>(staging + C::STAGING_BYTES);
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(swb) + C::SWB_BYTES);
     uint64_t* empty = full + C::STAGES;
-    uint64_t* conv = empty + C::STAGES;  // W8 / AQ: converted stage ready (arrivals from both CTAs' converters)
+    uint64_t* conv = empty + C::STAGES;  // W8: converted stage ready (arrivals from both CTAs' converters)
     uint64_t* tfull = conv + C::STAGES;
     uint64_t* tempty = tfull + C::ACC;
     uint64_t* drain = tempty + C::ACC;
     uint64_t* redbar = drain + 1;  // split-K: staged partial quarters landed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(redbar + 1);
+    uint64_t* qfull = redbar + 1;     // fused linear: a staged chunk of bf16 rows landed
+    uint64_t* qempty = qfull + kQgBufs;  // fused linear: a staging buffer is free again
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + kQgBufs);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile uint32_t* split_ticket = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);  // split-K
     volatile uint32_t* split_fail = reinterpret_cast<volatile uint32_t*>(tmem_slot + 3);    // split-K
     volatile uint32_t* split_ok = reinterpret_cast<volatile uint32_t*>(tmem_slot + 4);      // split-K
+    volatile int* qchunk = reinterpret_cast<volatile int*>(tmem_slot + 5);  // fused: chunk in each buffer [kQgBufs]
+    volatile int* qstate = reinterpret_cast<volatile int*>(tmem_slot + 8);  // fused: chunk being quantised
+    volatile uint32_t* qred = tmem_slot + 9;  // fused: [2][8] row maxima of the eight quantising warps
+    volatile uint32_t* qlast = tmem_slot + 25;  // fused: this CTA finished last
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -250,7 +278,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&conv[s], CG);  // the stage's converter warp in each CTA (W8 / AQ)
+            mbar_init(&conv[s], CG);  // the stage's converter warp in each CTA (W8)
         }
         for (int a = 0; a < C::ACC; ++a) {
             mbar_init(&tfull[a], 1);
@@ -258,6 +286,10 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
         }
         mbar_init(drain, 1);
         mbar_init(redbar, 1);
+        for (int b = 0; b < kQgBufs; ++b) {
+            mbar_init(&qfull[b], 1);
+            mbar_init(&qempty[b], 1);
+        }
         *abort_flag = 0;
         *split_ticket = 0u;
         *split_fail = 0u;
@@ -289,6 +321,115 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     pdl_wait();
     pdl_trigger();
 
+    if constexpr (C::QG) {
+        // ------------------------------------------------ phase Q (fused linear)
+        // Every CTA quantises rows of A until none are left unclaimed: thread
+        // 0 claims chunks of qg_rows rows in row order (one atomic per chunk)
+        // and bulk-copies each into one of kQgBufs staging buffers in the
+        // operand ring; the eight epilogue warps take each row's amax (threads
+        // per row qg_tpr, shuffles and, across warps, shared memory), its scale
+        // and its codes with the rowwise quantiser's arithmetic, store the
+        // codes and the scale, then count the chunk's rows as done for its
+        // 128-row block (release). A chunk is only ever claimed by a running
+        // CTA and nothing here waits on another CTA, so every counted row
+        // block completes; the GEMM below waits only for those counts.
+        if (warp == 0 && lane == 0) {
+            for (int it = 0;; ++it) {
+                const int b = it % kQgBufs;
+                if (!mbar_wait_bounded(&qempty[b], (uint32_t)((it / kQgBufs) & 1) ^ 1u, abort_flag, args.err)) {
+                    qchunk[b] = -1;
+                    mbar_arrive(&qfull[b]);
+                    break;
+                }
+                const int c = (int)atomicAdd(args.qg_ctr, 1u);
+                if (c >= args.qg_chunks) {
+                    qchunk[b] = -1;  // no rows left: the quantising warps stop at this buffer
+                    mbar_arrive(&qfull[b]);
+                    break;
+                }
+                const int r0 = c * args.qg_rows;
+                const int rows = args.M - r0 < args.qg_rows ? args.M - r0 : args.qg_rows;
+                const uint32_t bytes = (uint32_t)rows * (uint32_t)args.K * 2u;
+                qchunk[b] = c;
+                mbar_arrive_expect_tx(&qfull[b], bytes);
+                bulk_load_g2s(smem + (size_t)b * kQgBufBytes, args.qg_a + (size_t)r0 * args.K, bytes, &qfull[b]);
+            }
+        } else if (warp >= 2) {
+            const int qt = threadIdx.x - 64;  // 0..255
+            const int tpr = args.qg_tpr;
+            const int rpp = 256 / tpr;        // rows per pass
+            const int t = qt & (tpr - 1);
+            const int rr = qt / tpr;
+            const int nvec = args.K >> 3;
+            const int wpr = tpr >> 5;         // warps per row when tpr >= 32
+            for (int it = 0;; ++it) {
+                const int b = it % kQgBufs;
+                if (qt == 0) {
+                    const bool ok = mbar_wait_bounded(&qfull[b], (uint32_t)((it / kQgBufs) & 1), abort_flag, args.err);
+                    *qstate = ok ? qchunk[b] : -1;
+                }
+                named_barrier_sync(2, 256);
+                const int c = *qstate;
+                if (c < 0) break;  // uniform
+                const int r0 = c * args.qg_rows;
+                const int rows = args.M - r0 < args.qg_rows ? args.M - r0 : args.qg_rows;
+                const uint8_t* buf = smem + (size_t)b * kQgBufBytes;
+                for (int pass = 0; pass * rpp < rows; ++pass) {
+                    const int lr = pass * rpp + rr;  // row within the chunk
+                    const bool active = lr < rows;
+                    uint4 v[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int vi = i * tpr + t;
+                        v[i] = (active && vi < nvec)
+                                   ? *reinterpret_cast<const uint4*>(buf + (size_t)lr * args.K * 2 + (size_t)vi * 16)
+                                   : make_uint4(0, 0, 0, 0);
+                    }
+                    uint32_t packed = 0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) packed = absmax8(v[i], packed);
+                    uint32_t m = fold_halves(packed);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1)
+                        if (off < tpr) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+                    if (tpr > 32) {
+                        // Rows span wpr warps (tpr 64 .. 256): combine their maxima.
+                        volatile uint32_t* rb = qred + (pass & 1) * 8;
+                        if (lane == 0) rb[qt >> 5] = m;
+                        named_barrier_sync(2, 256);
+                        m = rb[rr * wpr];
+                        for (int w = 1; w < wpr; ++w) m = max(m, rb[rr * wpr + w]);
+                    }
+                    const ScaleCtx sc = scale_ctx<FP8DIT_E4M3FN>(bf16_bits_to_float(m));
+                    if (active) {
+                        const Quot2 q2 = quot2_of(sc);
+                        const int64_t row = (int64_t)r0 + lr;
+                        uint8_t* qrow = args.qg_q + row * args.K;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int vi = i * tpr + t;
+                            if (vi < nvec)
+                                *reinterpret_cast<uint2*>(qrow + (size_t)vi * 8) =
+                                    sc.fast ? quant8<FP8DIT_E4M3FN, true>(v[i], q2) : quant8<FP8DIT_E4M3FN, false>(v[i], q2);
+                        }
+                        if (t == 0) args.qg_s[row] = sc.s;
+                    }
+                }
+                // The chunk's codes and scales, then its count; the buffer goes
+                // back to thread 0 once every thread has read it.
+                __threadfence();
+                fence_proxy_async_smem();  // generic reads of the buffer before later async-proxy writes
+                named_barrier_sync(2, 256);
+                if (qt == 0) {
+                    red_add_release_gpu_u32(args.qg_ctr + 2 + (r0 >> 7), (uint32_t)rows);
+                    mbar_arrive(&qempty[b]);
+                }
+            }
+        }
+        // The operand ring is the GEMM's from here on.
+        __syncthreads();
+    }
+
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -300,6 +441,18 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 const TileCoord tc = tile_coord(args, sg.t);
                 const int a_row = tc.tm * C::BM + (int)rank * C::ROWS;
                 const int b_row = tc.tn * BN + (int)rank * C::B_ROWS;
+                if constexpr (C::QG) {
+                    // This CTA's 128 rows of A must be quantised (phase Q of
+                    // some running CTA) before their codes are loaded.
+                    const int need = args.M - a_row < C::ROWS ? args.M - a_row : C::ROWS;
+                    if (need > 0 && !wait_count_bounded(args.qg_ctr + 2 + (a_row >> 7), (uint32_t)need, abort_flag,
+                                                        args.err)) {
+                        aborted = true;
+                        abort_peer();
+                        break;
+                    }
+                    fence_proxy_async_global();  // the acquired codes, before the copies read them
+                }
                 for (int kb = sg.k0; kb < sg.k1; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, args.err)) {
                         aborted = true;
@@ -358,7 +511,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 for (int kb = sg.k0; kb < sg.k1; ++kb) {
-                    // W8 / AQ: both CTAs' converted operands (and, through the
+                    // W8: both CTAs' converted operands (and, through the
                     // converters' waits, both CTAs' loads) are ready. FP8: both
                     // CTAs' TMA loads landed.
                     if (!mbar_wait_bounded(CONV ? &conv[stage] : &full[stage], phase, abort_flag, args.err)) {
@@ -443,7 +596,9 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                              : make_uint4(0, 0, 0, 0);
             }
             const int row = tc.tm * C::BM + (int)rank * C::ROWS + q * 32 + lane;
-            p.sa = row < args.M ? (args.sa != nullptr ? __ldg(args.sa + row) : 1.0f) : 0.0f;
+            // Fused linear: the launch itself writes sa, so it is read after
+            // the tile's accumulator is ready (below), not ahead.
+            p.sa = (row < args.M && !C::QG) ? (args.sa != nullptr ? __ldg(args.sa + row) : 1.0f) : 0.0f;
         };
         auto publish = [&](const Pre& p) {  // this warp's smem copy of sw / bias (fp32)
 #pragma unroll
@@ -546,7 +701,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             const TileCoord tc = tile_coord(args, sg.t);
             __syncwarp();  // every lane is done reading the previous tile's copy
             publish(pre);
-            const float sa = pre.sa;
+            float sa = pre.sa;
             __syncwarp();
             if (has_next) fetch(nx.t, pre);
             const int row0 = tc.tm * C::BM + (int)rank * C::ROWS + q * 32;  // first row of this warp's box
@@ -602,6 +757,15 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 if (lane == 0) abort_peer();
                 if (!split) break;
                 failed = true;  // split-K: still meet the CTA's epilogue barriers below
+            }
+            if constexpr (C::QG) {
+                // This lane's row was counted as quantised before the producer
+                // loaded its codes; acquire that count here too, then read sa.
+                const int row = row0 + lane;
+                if (row < args.M) {
+                    (void)ld_acquire_gpu_u32(args.qg_ctr + 2 + (row >> 7));
+                    sa = __ldcg(args.sa + row);
+                }
             }
             tc_fence_after();
             const int n_tile = args.prob[tc.g].N;
@@ -813,77 +977,6 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 }
             }
         }
-        if constexpr (AQ) {
-            // ------------------------------------------------ bf16 -> FP8 A quantisers (AQ)
-            // Converter warp s owns ring stage s. The stage's A buffer holds
-            // the tile's ROWS x 128 bf16 as loaded (256-byte rows, unswizzled);
-            // each row is quantised with its token's scale sa[m] and
-            // reciprocal ra[m] (written by the scale pre-pass from the row
-            // amax, exactly as the rowwise quantiser derives them) by the same
-            // code path as the rowwise quantiser, so the codes are identical.
-            // They are written in place as ROWS rows x 128 codes with the
-            // 128-byte swizzle. Rows go in batches of 16, each read whole
-            // before any of it is written: FP8 rows [r0, r0 + 16) cover bf16
-            // rows [r0 / 2, r0 / 2 + 8), all read already (or, for r0 = 0, in
-            // this batch). Rows at or beyond M are zeros (TMA fill) and get
-            // scale 1.
-            constexpr int kIters = 8;                        // 16-byte bf16 chunks per lane per batch
-            constexpr int kRowsPerBatch = kIters * 32 / 16;  // 16 chunks per 256-byte bf16 row
-            const int own = warp - (2 + C::EPI_WARPS);
-            uint32_t stage = 0, phase = 0;
-            bool stop = false;
-            SegSched ss = seg_begin(args, unit, units, C::SPLIT_OK);
-            Segment sg;
-            while (!stop && seg_next(ss, sg)) {
-                const TileCoord tc = tile_coord(args, sg.t);
-                const int row_base = tc.tm * C::BM + (int)rank * C::ROWS;
-                for (int kb = sg.k0; kb < sg.k1; ++kb) {
-                    if ((int)stage == own) {
-                        const bool ok = mbar_wait_bounded(&full[stage], phase, abort_flag, args.err);
-                        if (!__all_sync(0xffffffffu, ok)) {
-                            if (lane == 0) abort_peer();
-                            stop = true;
-                            break;
-                        }
-                        uint8_t* buf = sA + stage * C::A_STAGE;
-#pragma unroll 1
-                        for (int r0 = 0; r0 < C::ROWS; r0 += kRowsPerBatch) {
-                            uint4 v[kIters];
-                            float sv[kIters], rv[kIters];
-#pragma unroll
-                            for (int i = 0; i < kIters; ++i) {
-                                const int idx = i * 32 + lane;  // chunk (idx & 15) of row r0 + (idx >> 4)
-                                v[i] = *reinterpret_cast<const uint4*>(buf + (r0 + (idx >> 4)) * 256 + (idx & 15) * 16);
-                                const int grow = row_base + r0 + (idx >> 4);
-                                sv[i] = grow < args.M ? __ldg(args.sa + grow) : 1.0f;
-                                rv[i] = grow < args.M ? __ldg(args.ra + grow) : 1.0f;
-                            }
-                            __syncwarp();  // the whole batch is read before any lane writes
-#pragma unroll
-                            for (int i = 0; i < kIters; ++i) {
-                                const int idx = i * 32 + lane;
-                                const int r = r0 + (idx >> 4), c16 = idx & 15;
-                                const Quot2 q2{f2_pack(rv[i], rv[i]), f2_pack(-sv[i], -sv[i]), sv[i]};
-                                const uint2 codes = rv[i] != 0.0f ? quant8<FP8DIT_E4M3FN, true>(v[i], q2)
-                                                                  : quant8<FP8DIT_E4M3FN, false>(v[i], q2);
-                                *reinterpret_cast<uint2*>(buf + r * 128 + (((c16 >> 1) ^ (r & 7)) << 4) +
-                                                          (c16 & 1) * 8) = codes;
-                            }
-                        }
-                        fence_proxy_async_smem();  // the tensor core reads these bytes through the async proxy
-                        __syncwarp();
-                        if (lane == 0) {
-                            if (CG == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&conv[stage]), 0));
-                            else mbar_arrive(&conv[stage]);
-                        }
-                    }
-                    if (++stage == C::STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-        }
         __syncwarp();
     }
 
@@ -896,6 +989,19 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (C::QG) {
+        // The CTA that finishes last returns the fused linear's counters to
+        // zero for the next launch (no other CTA reads them any more).
+        if (threadIdx.x == 0) {
+            __threadfence();
+            *qlast = atomicAdd(args.qg_ctr + 1, 1u) == gridDim.x - 1 ? 1u : 0u;
+        }
+        __syncthreads();
+        if (*qlast) {
+            const int nrb = (args.M + 127) >> 7;
+            for (int i = threadIdx.x; i < 2 + nrb; i += blockDim.x) args.qg_ctr[i] = 0u;
+        }
+    }
     if (CG == 2) cluster_sync_all();  // both CTAs done with TMEM and each other's barriers
     if (warp == 1) {
         tc_fence_after();
@@ -924,15 +1030,15 @@ cudaError_t launch_cfg(const GemmArgs& args, int units, cudaStream_t stream) {
 }  // namespace
 
 int gemm_cta_group(int cfg) {
-    return (cfg == kCfgPair256 || cfg == kCfgW8Pair256 || cfg == kCfgAQPair256) ? 2 : 1;
+    return (cfg == kCfgPair256 || cfg == kCfgW8Pair256 || cfg == kCfgQGPair256) ? 2 : 1;
 }
 int gemm_block_m(int cfg) { return 128 * gemm_cta_group(cfg); }
 int gemm_block_n(int cfg) {
-    return cfg == kCfg128x64 ? 64 : (cfg == kCfg128x128 || cfg == kCfgW8128x128 || cfg == kCfgAQ128x128) ? 128 : 256;
+    return cfg == kCfg128x64 ? 64 : (cfg == kCfg128x128 || cfg == kCfgW8128x128 || cfg == kCfgQG128x128) ? 128 : 256;
 }
 int gemm_b_box_rows(int cfg) { return cfg == kCfg128x256 ? 256 : cfg == kCfg128x64 ? 64 : 128; }
 bool gemm_weight_only(int cfg) { return cfg == kCfgW8Pair256 || cfg == kCfgW8128x128; }
-bool gemm_quantizes_a(int cfg) { return cfg == kCfgAQPair256 || cfg == kCfgAQ128x128; }
+bool gemm_quantizes_a(int cfg) { return cfg == kCfgQGPair256 || cfg == kCfgQG128x128; }
 int gemm_k_elems(int cfg) { return gemm_weight_only(cfg) ? 64 : 128; }
 
 // MMA units (CTA pairs or CTAs) to launch: one per tile, at most one per SM (pair).
@@ -953,10 +1059,10 @@ cudaError_t launch_gemm(int cfg, const GemmArgs& args, int units, cudaStream_t s
             return launch_cfg<2, 256, kOpsW8>(args, units, stream);
         case kCfgW8128x128:
             return launch_cfg<1, 128, kOpsW8>(args, units, stream);
-        case kCfgAQPair256:
-            return launch_cfg<2, 256, kOpsAQ>(args, units, stream);
-        case kCfgAQ128x128:
-            return launch_cfg<1, 128, kOpsAQ>(args, units, stream);
+        case kCfgQGPair256:
+            return launch_cfg<2, 256, kOpsQG>(args, units, stream);
+        case kCfgQG128x128:
+            return launch_cfg<1, 128, kOpsQG>(args, units, stream);
         case kCfg128x64:
             return launch_cfg<1, 64, kOpsFp8>(args, units, stream);
         default:

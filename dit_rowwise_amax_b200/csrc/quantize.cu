@@ -121,8 +121,7 @@ __device__ __forceinline__ void load_group(const uint16_t* __restrict__ x, int64
 template <int TPR, int VPT, int FMT, int ACT>
 __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* __restrict__ x, int64_t M,
                                                                  int32_t K, int64_t ldx, uint8_t* __restrict__ q,
-                                                                 int64_t ldq, float* __restrict__ scale,
-                                                                 float* __restrict__ rcp, int64_t groups,
+                                                                 int64_t ldq, float* __restrict__ scale, int64_t groups,
                                                                  uint16_t* __restrict__ gout, int64_t ldg) {
     constexpr int RPB = kThreads / TPR;
     constexpr int WPR = TPR / 32;  // warps per row (when TPR >= 32)
@@ -185,7 +184,7 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* _
         }
         const ScaleCtx c = scale_ctx<FMT>(bf16_bits_to_float(m));
         const int64_t row = g * RPB + r;
-        if (row < M && q != nullptr) {
+        if (row < M) {
             const Quot2 q2 = quot2_of(c);
             uint8_t* qr = q + row * ldq;
             if (c.fast) {
@@ -202,10 +201,7 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_regs(const uint16_t* _
                 }
             }
         }
-        if (row < M && t == 0) {
-            scale[row] = c.s;
-            if (rcp != nullptr) rcp[row] = c.fast ? c.r : 0.0f;
-        }
+        if (row < M && t == 0) scale[row] = c.s;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) cur[i] = nxt[i];
     }
@@ -218,7 +214,6 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_
                                                                      int64_t K, int64_t ldx,
                                                                      uint8_t* __restrict__ q, int64_t ldq,
                                                                      float* __restrict__ scale,
-                                                                     float* __restrict__ rcp,
                                                                      uint16_t* __restrict__ gout, int64_t ldg) {
     __shared__ uint32_t red[kThreads / 32];
     const int64_t nvec = K >> 3;
@@ -239,11 +234,7 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_
         for (int w = 1; w < kThreads / 32; ++w) m = max(m, red[w]);
         __syncthreads();  // red is reused by the next row
         const ScaleCtx c = scale_ctx<FMT>(bf16_bits_to_float(m));
-        if (threadIdx.x == 0) {
-            scale[row] = c.s;
-            if (rcp != nullptr) rcp[row] = c.fast ? c.r : 0.0f;
-        }
-        if (q == nullptr) continue;  // scales only
+        if (threadIdx.x == 0) scale[row] = c.s;
         const Quot2 q2 = quot2_of(c);
         uint8_t* qr = q + row * ldq;
         uint4* gr = gout != nullptr ? reinterpret_cast<uint4*>(gout + row * ldg) : nullptr;
@@ -258,10 +249,9 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_two_pass(const uint16_
 struct RowsArgs {
     const uint16_t* x;
     int64_t M, K, ldx;
-    uint8_t* q;  // null: scales only
+    uint8_t* q;
     int64_t ldq;
     float* scale;
-    float* rcp;  // optional: RN(1 / scale) where the corrected-reciprocal quotient applies, else 0
     uint16_t* g;
     int64_t ldg;
 };
@@ -279,7 +269,7 @@ cudaError_t launch_regs(const RowsArgs& a, cudaStream_t stream, const DeviceInfo
     const int64_t groups = (a.M + RPB - 1) / RPB;
     const int64_t grid = std::min<int64_t>(groups, (int64_t)dev->num_sms * per_sm);
     return launch_pdl(quantize_rows_regs<TPR, VPT, FMT, ACT>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1,
-                      a.x, a.M, (int32_t)a.K, a.ldx, a.q, a.ldq, a.scale, a.rcp, groups, a.g, a.ldg);
+                      a.x, a.M, (int32_t)a.K, a.ldx, a.q, a.ldq, a.scale, groups, a.g, a.ldg);
 }
 
 template <int FMT, int ACT>
@@ -288,7 +278,7 @@ cudaError_t launch_fmt(const RowsArgs& a, cudaStream_t stream, const DeviceInfo*
     if (nvec > 1024) {
         const int64_t grid = std::min<int64_t>(a.M, (int64_t)dev->num_sms * 8);
         return launch_pdl(quantize_rows_two_pass<FMT, ACT>, dim3((unsigned)grid), dim3(kThreads), 0, stream, 1, a.x,
-                          a.M, a.K, a.ldx, a.q, a.ldq, a.scale, a.rcp, a.g, a.ldg);
+                          a.M, a.K, a.ldx, a.q, a.ldq, a.scale, a.g, a.ldg);
     }
     // Smallest power-of-two group (>= 8 threads) that covers the row with <= 4 vectors each.
     int tpr = 8;
@@ -345,16 +335,9 @@ __global__ void selftest_quotient_kernel(unsigned long long* mismatch) {
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int fmt, uint8_t* q,
                                  int64_t ldq, float* scale, cudaStream_t stream, const DeviceInfo* dev) {
     if (M == 0) return cudaSuccess;
-    const RowsArgs a{x, M, K, ldx, q, ldq, scale, nullptr, nullptr, 0};
+    const RowsArgs a{x, M, K, ldx, q, ldq, scale, nullptr, 0};
     return fmt == FP8DIT_E4M3FN ? launch_fmt<FP8DIT_E4M3FN, 0>(a, stream, dev)
                                 : launch_fmt<FP8DIT_E5M2, 0>(a, stream, dev);
-}
-
-cudaError_t launch_row_scales(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float* scale, float* rcp,
-                              cudaStream_t stream, const DeviceInfo* dev) {
-    if (M == 0) return cudaSuccess;
-    const RowsArgs a{x, M, K, ldx, nullptr, 0, scale, rcp, nullptr, 0};
-    return launch_fmt<FP8DIT_E4M3FN, 0>(a, stream, dev);
 }
 
 // Builds the activation tables on the current device once (on `stream`, which
@@ -383,7 +366,7 @@ cudaError_t launch_act_quantize_rows(const uint16_t* h, int64_t M, int64_t K, in
     if (M == 0) return cudaSuccess;
     cudaError_t e = ensure_act_tables(stream);
     if (e != cudaSuccess) return e;
-    const RowsArgs a{h, M, K, ldh, q, ldq, scale, nullptr, g, ldg};
+    const RowsArgs a{h, M, K, ldh, q, ldq, scale, g, ldg};
     switch (act) {
         case FP8DIT_ACT_GELU_ERF:
             return launch_fmt<FP8DIT_E4M3FN, FP8DIT_ACT_GELU_ERF>(a, stream, dev);

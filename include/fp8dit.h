@@ -258,26 +258,33 @@ fp8dit_status fp8_weight_only_linear(fp8dit_linear h, int64_t M, const uint16_t*
                                      fp8dit_stream_t stream);
 
 /*
- * FP8 linear from a bf16 activation with the quantisation moved into the GEMM
- * (the fused variant of "从 BF16 到 FP8", section 三.1: runtime activation
- * quantisation feeding the FP8 GEMM). The per-token amax needs the whole row
- * before any element can be quantised, so a pre-pass reads A once and writes
- * per row the scale S = amax / 448 (1 for an all-zero row) and RN(1 / S) (0
- * where the exact-division quotient is used); the GEMM then loads bf16 tiles
- * of A and quantises them to E4M3 in shared memory next to the tensor cores.
- * The FP8 activation is never written to memory.
- * Result: the codes are the ones fp8_quantize_rowwise writes, so y equals what
- * fp8_scaled_linear computes from a_bf16 (bit for bit where both use 256 x 256
- * pair tiles; otherwise within the accumulation-order difference).
- *   a_bf16 [M, K] bf16 contiguous, 16-byte aligned;
- *   scale_scratch DEVICE float[2 * M], 4-byte aligned, caller-owned: the
- *     per-token scales S (first M) then their reciprocals; written by the call,
- *     S is left there for the caller;
- *   y [M, N] bf16 contiguous, 16-byte aligned.
- * M == 0 is a no-op. Must run on the handle's device.
+ * The FP8 linear from a bf16 activation in ONE launch (the fused variant of
+ * "从 BF16 到 FP8", section 三.1: runtime per-token activation quantisation
+ * feeding the FP8 GEMM; section 三.2 item 2: fewer extra reads and writes and
+ * intermediate launches). The launch's CTAs first quantise A together: each
+ * claims chunks of rows in row order, stages their bf16 values in shared
+ * memory with bulk copies, and writes each row's E4M3 codes and scale with
+ * the rowwise quantiser's arithmetic; every element is quantised exactly once.
+ * Each CTA then runs the FP8 GEMM + epilogue of fp8_scaled_linear, a tile
+ * starting as soon as its rows have been quantised. A chunk is only ever
+ * claimed by a running CTA and that work waits for nothing, so no wait
+ * depends on CTAs that have not started.
+ * Result: qa_scratch and sa_scratch hold exactly what fp8_quantize_rowwise
+ * writes, and y equals fp8_scaled_linear(h, M, a_bf16, ...) bit for bit where
+ * both use 256 x 256 pair tiles (otherwise within the accumulation-order
+ * difference of another tile plan).
+ *   a_bf16     [M, K] bf16 contiguous, 16-byte aligned;
+ *   qa_scratch [M, K] E4M3FN codes, 16-byte aligned, caller-owned: written;
+ *   sa_scratch [M] fp32 per-token scales, 4-byte aligned, caller-owned: written;
+ *   y          [M, N] bf16 contiguous, 16-byte aligned.
+ * The layer must have a workspace attached (fp8_linear_set_workspace): its
+ * counters, which every launch leaves at zero; calls that overlap on the GPU
+ * must not share it. Requires K <= 8192 and M <= 1048576
+ * (FP8DIT_ERR_UNSUPPORTED_SHAPE otherwise). M == 0 is a no-op. Must run on
+ * the handle's device.
  */
-fp8dit_status fp8_scaled_linear_fused(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, float* scale_scratch,
-                                      uint16_t* y, fp8dit_stream_t stream);
+fp8dit_status fp8_scaled_linear_fused(fp8dit_linear h, int64_t M, const uint16_t* a_bf16, uint8_t* qa_scratch,
+                                      float* sa_scratch, uint16_t* y, fp8dit_stream_t stream);
 
 /*
  * FP8 linear from HOST buffers, with the transfers pipelined around the

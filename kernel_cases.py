@@ -9,7 +9,7 @@ Cases (inputs from ``synth``, the same as the benchmark's):
     gelu_quantize_ffn_down               GELU -> E4M3 producer on a [4096, 8192] activation
     gemm_ffn_up, gemm_ffn_down           FP8 GEMM + epilogue from pre-quantised activations
     weight_only_ffn_up, ..._ffn_down     FP8 weight-only GEMM (bf16 activation)
-    fused_ffn_up, fused_ffn_down         quantise-in-GEMM variant (row-scale pre-pass + GEMM)
+    fused_ffn_up, fused_ffn_down         the fused linear (one launch: quantise, then GEMM)
     gemm_text_ffn_down                   FP8 GEMM, 26 tokens x FFN-down weight, plain schedule
     split_k_text_ffn_down                the same with a workspace attached (split-K schedule)
     weight_only_text_ffn_down            FP8 weight-only GEMM, 26 tokens x FFN-down weight
@@ -110,9 +110,11 @@ def run(case: str, iters: int) -> None:
             for _ in range(iters):
                 layer.forward_weight_only(a, y=y)
         else:
-            sc = torch.empty((2 * M,), dtype=torch.float32, device=dev)
+            qa = torch.empty((M, layer.K), dtype=torch.uint8, device=dev)
+            sa = torch.empty((M,), dtype=torch.float32, device=dev)
+            layer.attach_workspace()
             for _ in range(iters):
-                layer.forward_fused(a, y=y, scale_scratch=sc)
+                layer.forward_fused(a, y=y, qa_scratch=qa, sa_scratch=sa)
     torch.cuda.synchronize()
     if device_error() != 0:
         raise SystemExit(f"{case}: device error word set")

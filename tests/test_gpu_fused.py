@@ -1,13 +1,13 @@
-"""FP8 linear with the per-token quantisation inside the GEMM
-(fp8_scaled_linear_fused) on the GPU vs the CPU oracle.
+"""The FP8 linear from a bf16 activation in one launch (fp8_scaled_linear_fused)
+on the GPU vs the CPU oracle.
 
-The pre-pass's per-token scales must equal the oracle's bit for bit, and its
-reciprocals must be RN(1 / S) where the corrected-reciprocal quotient applies
-(amax >= 2^-64) and 0 elsewhere. The output is compared with the oracle's
-exact product of the oracle's own codes (|gpu - ref| <= 1e-2 |ref| +
-1e-3 rms(ref)), and, where both run 256 x 256 pair tiles, with the unfused
-fp8_scaled_linear bit for bit: the in-GEMM codes must be the rowwise
-quantiser's."""
+The launch's CTAs first quantise A per token (each element once) into the
+caller's scratch, then run the GEMM. The codes and scales it writes must equal
+the oracle's bit for bit; the output is compared with the oracle's exact
+product of the oracle's own codes (|gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref))
+and, where both run 256 x 256 pair tiles, with the two-launch
+fp8_scaled_linear bit for bit. Every launch must leave the workspace's
+counters at zero, so repeated calls and CUDA-graph replays need no reset."""
 
 import numpy as np
 import pytest
@@ -29,25 +29,17 @@ def make_layer(W, bias):
     return layer, qw.cpu().numpy(), sw.cpu().numpy()
 
 
-def expected_rcp(A, s):
-    """RN(1 / S) in fp32 where amax >= 2^-64, else 0."""
-    amax = np.abs(synth.bf16_to_f32(A)).max(axis=1)
-    with np.errstate(over="ignore"):  # 1 / S overflows only where the reciprocal is not used
-        r = (np.float32(1.0) / s).astype(np.float32)
-    return np.where(amax >= np.float32(2.0 ** -64), r, np.float32(0.0)).astype(np.float32)
-
-
 def run_fused(layer, A):
-    M = A.shape[0]
-    scratch = torch.empty((2 * M,), dtype=torch.float32, device="cuda")
-    y = layer.forward_fused(to_device_bf16(A), scale_scratch=scratch)
+    M, K = A.shape
+    qa = torch.full((M, K), 0xCD, dtype=torch.uint8, device="cuda")
+    sa = torch.full((M,), -1.0, dtype=torch.float32, device="cuda")
+    y = layer.forward_fused(to_device_bf16(A), qa_scratch=qa, sa_scratch=sa)
     torch.cuda.synchronize()
     assert fp8.device_error() == 0
-    qa, sa = oracle.quantize_rows(A, oracle.E4M3FN)
-    got = scratch.cpu().numpy()
-    assert np.array_equal(got[:M], sa), "per-token scales differ"
-    assert np.array_equal(got[M:], expected_rcp(A, sa)), "reciprocals differ"
-    return y, qa, sa
+    qo, so = oracle.quantize_rows(A, oracle.E4M3FN)
+    assert np.array_equal(sa.cpu().numpy().view(np.uint32), so.view(np.uint32)), "per-token scales differ"
+    assert np.array_equal(qa.cpu().numpy(), qo), "codes differ"
+    return y, qo, so
 
 
 def check_rows(y, qa, sa, qw, sw, bias, rows):
@@ -56,19 +48,25 @@ def check_rows(y, qa, sa, qw, sw, bias, rows):
     assert ok, f"tolerance exceeded: worst error / bound = {worst:.3f}"
 
 
+def counters_zero(layer):
+    ws = layer.workspace
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    flag_bytes = ws.numel() - pairs * 2 * 8 * 32 * 128 * 4  # everything before the fp32 partials
+    return int(torch.count_nonzero(ws[:flag_bytes])) == 0
+
+
 @pytest.mark.parametrize("cfg", ["ffn_up", "ffn_down"])
 def test_ffn_full_size_matches_unfused_bitwise(cfg):
     d = getattr(synth, cfg)()
     layer, qw, sw = make_layer(d["W"], d["bias"])
     M = d["A"].shape[0]
-    assert layer.plan(M)[:2] == (256, 256)
     y, qa, sa = run_fused(layer, d["A"])
+    layer.detach_workspace()
+    assert layer.plan(M)[:2] == (256, 256)
     y_ref = layer.forward(to_device_bf16(d["A"]))
     torch.cuda.synchronize()
     assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16)), "fused and unfused outputs differ"
-    rng = np.random.default_rng(3)
-    rows = np.unique(np.concatenate([np.arange(32), np.arange(M - 32, M), rng.integers(0, M, 32)]))
-    check_rows(y, qa, sa, qw, sw, d["bias"], rows)
+    check_rows(y, qa, sa, qw, sw, d["bias"], np.arange(M))
 
 
 def test_tiny_config_full():
@@ -76,10 +74,11 @@ def test_tiny_config_full():
     layer, qw, sw = make_layer(d["W"], d["bias"])
     y, qa, sa = run_fused(layer, d["A"])
     check_rows(y, qa, sa, qw, sw, d["bias"], np.arange(64))
+    assert counters_zero(layer)
 
 
 @pytest.mark.parametrize("M", [1, 26, 129, 257, 300])
-@pytest.mark.parametrize("N,K", [(8, 16), (136, 48), (520, 2064), (2048, 2048)])
+@pytest.mark.parametrize("N,K", [(8, 16), (136, 48), (520, 2064), (2048, 2048), (264, 8192)])
 def test_ragged_shapes(M, N, K):
     A = synth.normal_bf16(f"gpu/fused/A/{M}x{K}", (M, K), 1.0, outlier_p=0.01, outlier_factor=20.0)
     W = synth.normal_bf16(f"gpu/fused/W/{N}x{K}", (N, K), 0.02)
@@ -87,12 +86,13 @@ def test_ragged_shapes(M, N, K):
     layer, qw, sw = make_layer(W, bias)
     y, qa, sa = run_fused(layer, A)
     check_rows(y, qa, sa, qw, sw, bias, np.arange(M))
+    assert counters_zero(layer)
 
 
 def test_special_rows():
     """All-zero and all -0 rows (S = 1), a constant row, rows whose amax is
-    below 2^-64 (exact-division quotient, reciprocal 0), bf16 subnormals, in a
-    ragged 300 x 2064 activation spanning two pair tiles."""
+    below 2^-64 (exact-division quotient), bf16 subnormals, in a ragged
+    300 x 2064 activation spanning two pair tiles."""
     M, N, K = 300, 264, 2064
     A = synth.normal_bf16("gpu/fused/special/A", (M, K), 1.0, outlier_p=0.01, outlier_factor=30.0).copy()
     A[0] = 0x0000                       # +0
@@ -111,31 +111,80 @@ def test_special_rows():
     check_rows(y, qa, sa, qw, sw, bias, np.arange(M))
 
 
+def test_repeated_calls_and_graph_replays():
+    """Stream-ordered calls and replays of a captured graph, with new inputs
+    between replays: every result equals the first call's for the same input,
+    and the counters are back at zero after each."""
+    M, N, K = 1000, 2048, 2048
+    W = synth.normal_bf16("gpu/fused/graph/W", (N, K), 0.02)
+    layer, _, _ = make_layer(W, synth.normal_bf16("gpu/fused/graph/b", (N,), 0.1))
+    As = [to_device_bf16(synth.normal_bf16(f"gpu/fused/graph/A{i}", (M, K), 1.0)) for i in range(3)]
+    refs = [layer.forward_fused(a) for a in As]
+    torch.cuda.synchronize()
+    assert counters_zero(layer)
+    for _ in range(2):
+        for a, r in zip(As, refs):
+            assert torch.equal(layer.forward_fused(a).view(torch.int16), r.view(torch.int16))
+    a_in = As[0].clone()
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    qa = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    sa = torch.empty((M,), dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer.forward_fused(a_in, y=y, qa_scratch=qa, sa_scratch=sa)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.forward_fused(a_in, y=y, qa_scratch=qa, sa_scratch=sa)
+    for i in (1, 2, 0):
+        a_in.copy_(As[i])
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y.view(torch.int16), refs[i].view(torch.int16)), f"replay with input {i}"
+    del g
+    assert fp8.device_error() == 0
+    assert counters_zero(layer)
+
+
 def test_argument_errors_launch_nothing():
     L = fp8.load_library()
     W = synth.normal_bf16("gpu/fused/err/W", (64, 128), 0.02)
     layer, _, _ = make_layer(W, None)
     a = to_device_bf16(synth.normal_bf16("gpu/fused/err/A", (16, 128), 1.0))
-    y = torch.empty((16, 64), dtype=torch.bfloat16, device="cuda")
-    sc = torch.empty((64,), dtype=torch.float32, device="cuda")
+    y = torch.full((16, 64), 3.0, dtype=torch.bfloat16, device="cuda")
+    qa = torch.empty((16, 128), dtype=torch.uint8, device="cuda")
+    sa = torch.empty((16,), dtype=torch.float32, device="cuda")
     s = fp8._stream(a.device)
-    assert L.fp8_scaled_linear_fused(layer.handle, 16, a.data_ptr(), None, y.data_ptr(), s) == 1
-    assert L.fp8_scaled_linear_fused(layer.handle, 16, a.data_ptr(), sc.data_ptr() + 2, y.data_ptr(), s) == 1
-    assert L.fp8_scaled_linear_fused(layer.handle, 16, a.data_ptr() + 8, sc.data_ptr(), y.data_ptr(), s) == 1
-    assert L.fp8_scaled_linear_fused(layer.handle, -1, a.data_ptr(), sc.data_ptr(), y.data_ptr(), s) == 1
-    assert L.fp8_scaled_linear_fused(layer.handle, 0, None, None, None, s) == 0
-    assert L.fp8_scaled_linear_fused(None, 16, a.data_ptr(), sc.data_ptr(), y.data_ptr(), s) == 1
+    # No workspace attached yet: refused.
+    assert L.fp8_scaled_linear_fused(layer.handle, 16, a.data_ptr(), qa.data_ptr(), sa.data_ptr(), y.data_ptr(), s) == 1
+    layer.attach_workspace()
+    assert L.fp8_scaled_linear_fused(layer.handle, 16, a.data_ptr(), None, sa.data_ptr(), y.data_ptr(), s) == 1
+    assert L.fp8_scaled_linear_fused(layer.handle, 16, a.data_ptr(), qa.data_ptr(), sa.data_ptr() + 2, y.data_ptr(), s) == 1
+    assert L.fp8_scaled_linear_fused(layer.handle, 16, a.data_ptr() + 8, qa.data_ptr(), sa.data_ptr(), y.data_ptr(), s) == 1
+    assert L.fp8_scaled_linear_fused(layer.handle, 16, a.data_ptr(), qa.data_ptr() + 8, sa.data_ptr(), y.data_ptr(), s) == 1
+    assert L.fp8_scaled_linear_fused(layer.handle, -1, a.data_ptr(), qa.data_ptr(), sa.data_ptr(), y.data_ptr(), s) == 1
+    assert L.fp8_scaled_linear_fused(layer.handle, 0, None, None, None, None, s) == 0
+    assert L.fp8_scaled_linear_fused(None, 16, a.data_ptr(), qa.data_ptr(), sa.data_ptr(), y.data_ptr(), s) == 1
     torch.cuda.synchronize()
+    assert bool(torch.all(y == 3.0)), "a refused call wrote its output"
     assert fp8.device_error() == 0
 
 
-@pytest.mark.parametrize("M,N,K", [(200, 264, 16384), (37, 24, 8208)])
-def test_long_rows_two_pass_scale_prepass(M, N, K):
-    """Rows longer than 8192 elements take the two-pass row-scale pre-pass
-    (scales only, no codes written)."""
-    A = synth.normal_bf16(f"gpu/fused/long/A/{M}x{K}", (M, K), 1.0, outlier_p=0.01, outlier_factor=20.0)
-    W = synth.normal_bf16(f"gpu/fused/long/W/{N}x{K}", (N, K), 0.02)
-    bias = synth.normal_bf16(f"gpu/fused/long/b/{N}", (N,), 0.1)
-    layer, qw, sw = make_layer(W, bias)
-    y, qa, sa = run_fused(layer, A)
-    check_rows(y, qa, sa, qw, sw, bias, np.arange(M))
+def test_long_rows_refused():
+    """Rows longer than 8192 elements do not fit the launch's staging: refused
+    with UNSUPPORTED_SHAPE, nothing written."""
+    L = fp8.load_library()
+    M, N, K = 8, 64, 8208
+    layer, _, _ = make_layer(synth.normal_bf16("gpu/fused/long/W", (N, K), 0.02), None)
+    layer.attach_workspace()
+    a = to_device_bf16(synth.normal_bf16("gpu/fused/long/A", (M, K), 1.0))
+    y = torch.full((M, N), 3.0, dtype=torch.bfloat16, device="cuda")
+    qa = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    sa = torch.empty((M,), dtype=torch.float32, device="cuda")
+    st = L.fp8_scaled_linear_fused(layer.handle, M, a.data_ptr(), qa.data_ptr(), sa.data_ptr(), y.data_ptr(),
+                                   fp8._stream(a.device))
+    assert st == 2
+    torch.cuda.synchronize()
+    assert bool(torch.all(y == 3.0))

@@ -88,13 +88,14 @@ def test_multi_act_weight_only_and_fused():
     sh = torch.empty((M,), dtype=torch.float32, device="cuda")
     yw = torch.empty((M, 512), dtype=torch.bfloat16, device="cuda")
     yf = torch.empty((M, 512), dtype=torch.bfloat16, device="cuda")
-    sc = torch.empty((2 * M,), dtype=torch.float32, device="cuda")
+    qf = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+    sf = torch.empty((M,), dtype=torch.float32, device="cuda")
     fp8.act_quantize_rowwise(a, "gelu")  # builds the activation tables (synchronises once) before capture
 
     def run():
         fp8.scaled_linear_multi(layers, a, ys=ys, qa_scratch=qa, sa_scratch=sa)
         fp8.act_quantize_rowwise(a, "gelu", q=qh, scale=sh)
         layers[0].forward_weight_only(a, y=yw)
-        layers[2].forward_fused(a, y=yf, scale_scratch=sc)
+        layers[2].forward_fused(a, y=yf, qa_scratch=qf, sa_scratch=sf)
 
-    check_replays(lambda i: [rand_bf16(f"gpu/graph/B{i}", (M, K))], [a], run, ys + [qh, sh, yw, yf])
+    check_replays(lambda i: [rand_bf16(f"gpu/graph/B{i}", (M, K))], [a], run, ys + [qh, sh, yw, yf, qf, sf])

@@ -1,5 +1,5 @@
 """Seeded random shapes through the three linear paths (the FP8 linear from a
-bf16 activation, the FP8 weight-only linear, the quantise-in-GEMM variant),
+bf16 activation, the FP8 weight-only linear, the fused one-launch linear),
 each compared elementwise with the oracle on every output. The shapes mix
 every tile plan (pair tiles, 128 x 256, 128 x 128, 128 x 64), ragged M, N and
 K, and short K (a single k-block) to K = 4096. A second set of few-row shapes
