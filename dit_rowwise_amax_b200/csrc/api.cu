@@ -318,19 +318,13 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
     }
     args.sa = sa;
     if (qg != nullptr) {
-        // Rows per staged chunk: a power of two dividing 128 whose bf16 rows
-        // fit one staging buffer; threads per row: the smallest power of two
-        // (8 .. 256) that covers a row with at most four 16-byte vectors each.
-        int rows = 128;
-        while (rows > 1 && (uint64_t)rows * (uint64_t)K * 2 > kQgBufBytes) rows >>= 1;
-        int tpr = 8;
-        while (tpr * 4 < K / 8) tpr *= 2;
+        // Rows per staged chunk: as many bf16 rows as fit one staging buffer.
+        const int rows = (int)(kQgBufBytes / ((uint32_t)K * 2u));
         args.qg_a = qg->a;
         args.qg_q = qg->qa;
         args.qg_s = qg->sa;
         args.qg_ctr = static_cast<uint32_t*>(hs[0]->sk_ws) + qg_offset_words(hs[0]->num_sms / 2);
         args.qg_rows = rows;
-        args.qg_tpr = tpr;
         args.qg_chunks = (int32_t)((M + rows - 1) / rows);
     }
     args.M = (int32_t)M;

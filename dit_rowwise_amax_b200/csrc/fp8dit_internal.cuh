@@ -120,8 +120,7 @@ struct alignas(64) GemmArgs {
     uint8_t* qg_q;         // its E4M3 codes [M, K] (what tmA describes)
     float* qg_s;           // its per-token scales [M] (== sa)
     uint32_t* qg_ctr;      // [0] chunks claimed, [1] CTAs finished, [2 + b] rows of 128-row block b quantised
-    int32_t qg_rows;       // rows per chunk (a power of two dividing 128; rows x K x 2 <= kQgBufBytes)
-    int32_t qg_tpr;        // threads per row (power of two, 8..256) in the quantising warps
+    int32_t qg_rows;       // rows per chunk (rows x K x 2 <= kQgBufBytes)
     int32_t qg_chunks;     // ceil(M / qg_rows)
     uint32_t* sk_flag;   // stream-K: [units + 1][2 CTAs][8 epilogue warps] (zero between launches)
     float* sk_partial;   // stream-K: [units][2 CTAs][8 epilogue warps][32 rows][128 columns];
@@ -141,11 +140,12 @@ struct alignas(64) GemmArgs {
 constexpr size_t kSkFlagBytesPerUnit = 2 * 8 * sizeof(uint32_t);
 inline size_t sk_flag_words(int units) { return (size_t)(units + 1) * 16; }
 inline size_t split_flag_offset_words(int units) { return sk_flag_words(units); }
-// Fused linear: rows are quantised in chunks staged in shared memory, at most
-// kQgBufs chunks of kQgBufBytes in flight per CTA; readiness is counted per
-// 128-row block, so M <= 128 x kQgMaxRowBlocks; rows up to kQgMaxK elements.
-constexpr int kQgBufs = 3;
-constexpr uint32_t kQgBufBytes = 65536;
+// Fused linear: rows are quantised in chunks staged in shared memory, one
+// staging buffer of kQgBufBytes per quantising warp (kQgBufs of them);
+// readiness is counted per 128-row block, so M <= 128 x kQgMaxRowBlocks;
+// rows up to kQgMaxK elements (one row must fit a buffer).
+constexpr int kQgBufs = 8;
+constexpr uint32_t kQgBufBytes = 24576;
 constexpr int kQgMaxRowBlocks = 8192;
 constexpr int kQgMaxK = 8192;
 inline size_t qg_offset_words(int units) { return split_flag_offset_words(units) + 2 * (size_t)units; }

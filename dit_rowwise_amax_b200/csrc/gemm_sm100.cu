@@ -106,7 +106,7 @@ struct Cfg {
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_SMEM + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
     static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-    static_assert((3 * STAGES + 2 * ACC + 2 + 2 * kQgBufs) * 8 + 4 * 32 <= BAR_BYTES, "barrier area");
+    static_assert((3 * STAGES + 2 * ACC + 2 + 2 * kQgBufs) * 8 + 4 * (6 + kQgBufs) <= BAR_BYTES, "barrier area");
     // Fused linear: kQgBufs chunks of bf16 rows (kQgBufBytes each) are staged
     // in the operand ring before the GEMM uses it.
     static_assert(!QG || kQgBufs * kQgBufBytes <= STAGES * STAGE_SMEM, "quantiser staging");
@@ -258,9 +258,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     volatile uint32_t* split_fail = reinterpret_cast<volatile uint32_t*>(tmem_slot + 3);    // split-K
     volatile uint32_t* split_ok = reinterpret_cast<volatile uint32_t*>(tmem_slot + 4);      // split-K
     volatile int* qchunk = reinterpret_cast<volatile int*>(tmem_slot + 5);  // fused: chunk in each buffer [kQgBufs]
-    volatile int* qstate = reinterpret_cast<volatile int*>(tmem_slot + 8);  // fused: chunk being quantised
-    volatile uint32_t* qred = tmem_slot + 9;  // fused: [2][8] row maxima of the eight quantising warps
-    volatile uint32_t* qlast = tmem_slot + 25;  // fused: this CTA finished last
+    volatile uint32_t* qlast = tmem_slot + 5 + kQgBufs;  // fused: this CTA finished last
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -323,106 +321,88 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
 
     if constexpr (C::QG) {
         // ------------------------------------------------ phase Q (fused linear)
-        // Every CTA quantises rows of A until none are left unclaimed: thread
-        // 0 claims chunks of qg_rows rows in row order (one atomic per chunk)
-        // and bulk-copies each into one of kQgBufs staging buffers in the
-        // operand ring; the eight epilogue warps take each row's amax (threads
-        // per row qg_tpr, shuffles and, across warps, shared memory), its scale
-        // and its codes with the rowwise quantiser's arithmetic, store the
-        // codes and the scale, then count the chunk's rows as done for its
-        // 128-row block (release). A chunk is only ever claimed by a running
-        // CTA and nothing here waits on another CTA, so every counted row
-        // block completes; the GEMM below waits only for those counts.
+        // Every CTA quantises rows of A until none are left unclaimed. Thread
+        // 0 claims chunks of qg_rows rows in row order (one atomic per chunk,
+        // issued one chunk ahead) and bulk-copies chunk i of this CTA into
+        // staging buffer i mod 8 in the operand ring. Quantising warp w owns
+        // buffer w: for each of its chunks it takes the rows one at a time, a
+        // sweep over the row in shared memory for its amax (shuffles), its
+        // scale, then a second sweep that writes its codes with the rowwise
+        // quantiser's arithmetic; after the chunk it counts the rows as done
+        // for their 128-row blocks (release) and hands the buffer back. No
+        // warp waits for another warp's rows and nothing here waits on another
+        // CTA; a chunk is only ever claimed by a running CTA, so every counted
+        // row block completes, and the GEMM below waits only for those counts.
         if (warp == 0 && lane == 0) {
-            for (int it = 0;; ++it) {
+            const int R = args.qg_rows;
+            int c = (int)atomicAdd(args.qg_ctr, 1u);
+            int stop = 0;  // buffers that have been given the end mark
+            for (int it = 0; stop < kQgBufs; ++it) {
                 const int b = it % kQgBufs;
                 if (!mbar_wait_bounded(&qempty[b], (uint32_t)((it / kQgBufs) & 1) ^ 1u, abort_flag, args.err)) {
-                    qchunk[b] = -1;
-                    mbar_arrive(&qfull[b]);
+                    // Give up: mark every buffer, waiting for none of them.
+                    for (int k = 0; k < kQgBufs; ++k) qchunk[k] = -1;
+                    for (int k = 0; k < kQgBufs; ++k) mbar_arrive(&qfull[k]);
                     break;
                 }
-                const int c = (int)atomicAdd(args.qg_ctr, 1u);
                 if (c >= args.qg_chunks) {
-                    qchunk[b] = -1;  // no rows left: the quantising warps stop at this buffer
+                    qchunk[b] = -1;  // no rows left: warp b stops at this buffer
                     mbar_arrive(&qfull[b]);
-                    break;
+                    ++stop;
+                    continue;
                 }
-                const int r0 = c * args.qg_rows;
-                const int rows = args.M - r0 < args.qg_rows ? args.M - r0 : args.qg_rows;
+                const int r0 = c * R;
+                const int rows = args.M - r0 < R ? args.M - r0 : R;
                 const uint32_t bytes = (uint32_t)rows * (uint32_t)args.K * 2u;
                 qchunk[b] = c;
                 mbar_arrive_expect_tx(&qfull[b], bytes);
                 bulk_load_g2s(smem + (size_t)b * kQgBufBytes, args.qg_a + (size_t)r0 * args.K, bytes, &qfull[b]);
+                c = (int)atomicAdd(args.qg_ctr, 1u);  // the next claim, in flight while this buffer fills
             }
         } else if (warp >= 2) {
-            const int qt = threadIdx.x - 64;  // 0..255
-            const int tpr = args.qg_tpr;
-            const int rpp = 256 / tpr;        // rows per pass
-            const int t = qt & (tpr - 1);
-            const int rr = qt / tpr;
-            const int nvec = args.K >> 3;
-            const int wpr = tpr >> 5;         // warps per row when tpr >= 32
-            for (int it = 0;; ++it) {
-                const int b = it % kQgBufs;
-                if (qt == 0) {
-                    const bool ok = mbar_wait_bounded(&qfull[b], (uint32_t)((it / kQgBufs) & 1), abort_flag, args.err);
-                    *qstate = ok ? qchunk[b] : -1;
-                }
-                named_barrier_sync(2, 256);
-                const int c = *qstate;
-                if (c < 0) break;  // uniform
-                const int r0 = c * args.qg_rows;
-                const int rows = args.M - r0 < args.qg_rows ? args.M - r0 : args.qg_rows;
-                const uint8_t* buf = smem + (size_t)b * kQgBufBytes;
-                for (int pass = 0; pass * rpp < rows; ++pass) {
-                    const int lr = pass * rpp + rr;  // row within the chunk
-                    const bool active = lr < rows;
-                    uint4 v[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int vi = i * tpr + t;
-                        v[i] = (active && vi < nvec)
-                                   ? *reinterpret_cast<const uint4*>(buf + (size_t)lr * args.K * 2 + (size_t)vi * 16)
-                                   : make_uint4(0, 0, 0, 0);
-                    }
+            const int w = warp - 2;  // owns staging buffer w
+            const int R = args.qg_rows;
+            const int K = args.K;
+            const int nvec = K >> 3;
+            for (int j = 0;; ++j) {
+                const bool ok = mbar_wait_bounded(&qfull[w], (uint32_t)(j & 1), abort_flag, args.err);
+                const int c = ok ? qchunk[w] : -1;
+                if (!__all_sync(0xffffffffu, c >= 0)) break;  // no more rows (or an expired wait)
+                const int r0 = c * R;
+                const int rows = args.M - r0 < R ? args.M - r0 : R;
+                for (int lr = 0; lr < rows; ++lr) {
+                    const int64_t row = (int64_t)r0 + lr;
+                    const uint4* src =
+                        reinterpret_cast<const uint4*>(smem + (size_t)w * kQgBufBytes + (size_t)lr * K * 2);
                     uint32_t packed = 0;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) packed = absmax8(v[i], packed);
+                    for (int vi = lane; vi < nvec; vi += 32) packed = absmax8(src[vi], packed);
                     uint32_t m = fold_halves(packed);
 #pragma unroll
-                    for (int off = 16; off > 0; off >>= 1)
-                        if (off < tpr) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
-                    if (tpr > 32) {
-                        // Rows span wpr warps (tpr 64 .. 256): combine their maxima.
-                        volatile uint32_t* rb = qred + (pass & 1) * 8;
-                        if (lane == 0) rb[qt >> 5] = m;
-                        named_barrier_sync(2, 256);
-                        m = rb[rr * wpr];
-                        for (int w = 1; w < wpr; ++w) m = max(m, rb[rr * wpr + w]);
-                    }
+                    for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
                     const ScaleCtx sc = scale_ctx<FP8DIT_E4M3FN>(bf16_bits_to_float(m));
-                    if (active) {
-                        const Quot2 q2 = quot2_of(sc);
-                        const int64_t row = (int64_t)r0 + lr;
-                        uint8_t* qrow = args.qg_q + row * args.K;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int vi = i * tpr + t;
-                            if (vi < nvec)
-                                *reinterpret_cast<uint2*>(qrow + (size_t)vi * 8) =
-                                    sc.fast ? quant8<FP8DIT_E4M3FN, true>(v[i], q2) : quant8<FP8DIT_E4M3FN, false>(v[i], q2);
-                        }
-                        if (t == 0) args.qg_s[row] = sc.s;
+                    const Quot2 q2 = quot2_of(sc);
+                    uint2* dst = reinterpret_cast<uint2*>(args.qg_q + row * K);
+                    if (sc.fast) {
+                        for (int vi = lane; vi < nvec; vi += 32) dst[vi] = quant8<FP8DIT_E4M3FN, true>(src[vi], q2);
+                    } else {
+                        for (int vi = lane; vi < nvec; vi += 32) dst[vi] = quant8<FP8DIT_E4M3FN, false>(src[vi], q2);
                     }
+                    if (lane == 0) args.qg_s[row] = sc.s;
                 }
-                // The chunk's codes and scales, then its count; the buffer goes
-                // back to thread 0 once every thread has read it.
+                // The chunk's codes and scales, then its counts; the staged rows
+                // have been read (generic proxy) before the copy engine (async
+                // proxy) refills the buffer.
                 __threadfence();
-                fence_proxy_async_smem();  // generic reads of the buffer before later async-proxy writes
-                named_barrier_sync(2, 256);
-                if (qt == 0) {
-                    red_add_release_gpu_u32(args.qg_ctr + 2 + (r0 >> 7), (uint32_t)rows);
-                    mbar_arrive(&qempty[b]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    for (int r = r0; r < r0 + rows;) {
+                        const int blk = r >> 7;
+                        const int e = (blk + 1) * 128 < r0 + rows ? (blk + 1) * 128 : r0 + rows;
+                        red_add_release_gpu_u32(args.qg_ctr + 2 + blk, (uint32_t)(e - r));
+                        r = e;
+                    }
+                    mbar_arrive(&qempty[w]);
                 }
             }
         }
