@@ -146,6 +146,7 @@ inline size_t split_flag_offset_words(int units) { return sk_flag_words(units); 
 // rows up to kQgMaxK elements (one row must fit a buffer).
 constexpr int kQgBufs = 8;
 constexpr uint32_t kQgBufBytes = 24576;
+constexpr int kQgClaim = 4;  // chunks claimed per atomic (even, >= 2)
 constexpr int kQgMaxRowBlocks = 8192;
 constexpr int kQgMaxK = 8192;
 inline size_t qg_offset_words(int units) { return split_flag_offset_words(units) + 2 * (size_t)units; }

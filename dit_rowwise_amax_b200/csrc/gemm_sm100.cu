@@ -322,8 +322,8 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     if constexpr (C::QG) {
         // ------------------------------------------------ phase Q (fused linear)
         // Every CTA quantises rows of A until none are left unclaimed. Thread
-        // 0 claims chunks of qg_rows rows in row order (one atomic per chunk,
-        // issued one chunk ahead) and bulk-copies chunk i of this CTA into
+        // 0 claims chunks of qg_rows rows in row order (kQgClaim chunks per
+        // atomic) and bulk-copies chunk i of this CTA into
         // staging buffer i mod 8 in the operand ring. Quantising warp w owns
         // buffer w: for each of its chunks it takes the rows one at a time, a
         // sweep over the row in shared memory for its amax (shuffles), its
@@ -335,16 +335,22 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
         // row block completes, and the GEMM below waits only for those counts.
         if (warp == 0 && lane == 0) {
             const int R = args.qg_rows;
-            int c = (int)atomicAdd(args.qg_ctr, 1u);
-            int stop = 0;  // buffers that have been given the end mark
+            // Chunks are claimed kQgClaim at a time; the next batch is claimed
+            // halfway through staging the current one, so the atomic's round
+            // trip overlaps the copies.
+            int cur = (int)atomicAdd(args.qg_ctr, (uint32_t)kQgClaim);
+            int nxt = 0;
+            int k = 0;      // chunks of the current batch staged so far
+            int stop = 0;   // buffers that have been given the end mark
             for (int it = 0; stop < kQgBufs; ++it) {
                 const int b = it % kQgBufs;
                 if (!mbar_wait_bounded(&qempty[b], (uint32_t)((it / kQgBufs) & 1) ^ 1u, abort_flag, args.err)) {
                     // Give up: mark every buffer, waiting for none of them.
-                    for (int k = 0; k < kQgBufs; ++k) qchunk[k] = -1;
-                    for (int k = 0; k < kQgBufs; ++k) mbar_arrive(&qfull[k]);
+                    for (int q = 0; q < kQgBufs; ++q) qchunk[q] = -1;
+                    for (int q = 0; q < kQgBufs; ++q) mbar_arrive(&qfull[q]);
                     break;
                 }
+                const int c = cur + k;
                 if (c >= args.qg_chunks) {
                     qchunk[b] = -1;  // no rows left: warp b stops at this buffer
                     mbar_arrive(&qfull[b]);
@@ -357,7 +363,11 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 qchunk[b] = c;
                 mbar_arrive_expect_tx(&qfull[b], bytes);
                 bulk_load_g2s(smem + (size_t)b * kQgBufBytes, args.qg_a + (size_t)r0 * args.K, bytes, &qfull[b]);
-                c = (int)atomicAdd(args.qg_ctr, 1u);  // the next claim, in flight while this buffer fills
+                if (++k == kQgClaim / 2) nxt = (int)atomicAdd(args.qg_ctr, (uint32_t)kQgClaim);
+                if (k == kQgClaim) {
+                    cur = nxt;
+                    k = 0;
+                }
             }
         } else if (warp >= 2) {
             const int w = warp - 2;  // owns staging buffer w
