@@ -385,6 +385,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                     const uint4* src =
                         reinterpret_cast<const uint4*>(smem + (size_t)w * kQgBufBytes + (size_t)lr * K * 2);
                     uint32_t packed = 0;
+#pragma unroll 4
                     for (int vi = lane; vi < nvec; vi += 32) packed = absmax8(src[vi], packed);
                     uint32_t m = fold_halves(packed);
 #pragma unroll
@@ -393,6 +394,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                     const Quot2 q2 = quot2_of(sc);
                     uint2* dst = reinterpret_cast<uint2*>(args.qg_q + row * K);
                     if (sc.fast) {
+#pragma unroll 4
                         for (int vi = lane; vi < nvec; vi += 32) dst[vi] = quant8<FP8DIT_E4M3FN, true>(src[vi], q2);
                     } else {
                         for (int vi = lane; vi < nvec; vi += 32) dst[vi] = quant8<FP8DIT_E4M3FN, false>(src[vi], q2);
