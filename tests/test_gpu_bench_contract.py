@@ -54,8 +54,10 @@ def test_bench_json_line():
         for key in ("linear_us", "linear_tflops", "linear_frac", "quantize_us", "gemm_us", "gemm_frac"):
             assert t[layer][key] > 0, (layer, key)
         M, N, K = (4096, 8192, 2048) if layer == "ffn_up" else (4096, 2048, 8192)
-        assert t[layer]["linear_tflops"] == pytest.approx(2.0 * M * N * K / (t[layer]["linear_us"] * 1e-6) / 1e12)
-        assert t[layer]["linear_frac"] == pytest.approx(t[layer]["linear_tflops"] / t["peaks"]["fp8_tflops"])
+        # (the per-target figures are rounded to four significant digits)
+        assert t[layer]["linear_tflops"] == pytest.approx(2.0 * M * N * K / (t[layer]["linear_us"] * 1e-6) / 1e12,
+                                                          rel=2e-3)
+        assert t[layer]["linear_frac"] == pytest.approx(t[layer]["linear_tflops"] / t["peaks"]["fp8_tflops"], rel=2e-3)
     for key in ("ffn_up_gbs", "ffn_up_frac", "ffn_down_gbs", "ffn_down_frac"):
         assert t["quantizer"][key] > 0, key
-    assert rf["linear_ffn_up_frac"] == pytest.approx(t["ffn_up"]["linear_frac"])
+    assert rf["linear_ffn_up_frac"] == pytest.approx(t["ffn_up"]["linear_frac"], rel=2e-3)
