@@ -762,13 +762,12 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             tc_fence_after();
             const int n_tile = args.prob[tc.g].N;
             const uint32_t t_addr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + col0;
-#pragma unroll 1
-            for (int c = 0; c < (failed ? 0 : C::EPI_COLS / 32); ++c) {
-                const int n0 = tc.tn * BN + col0 + c * 32;
-                if (n0 >= n_tile) break;  // warp-uniform
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(t_addr + c * 32, r);
-                tmem_wait_ld();
+            // One 16-column half of 32-column chunk c, its accumulator in r:
+            // split-K and stream-K tails store it raw; otherwise (a stream-K
+            // head first adds its partner's partial) scale, bias, bf16 and
+            // half of row `lane` of the chunk's 32 x 32 staging box (64-byte
+            // rows, 64-byte swizzle).
+            auto half = [&](int c, int hh, uint32_t(&r)[16]) {
                 if (split) {
                     // This piece's raw fp32 partial, [q][column part][float4][lane]:
                     // every warp store moves 512 contiguous bytes. Warps whose
@@ -776,43 +775,39 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                     if (row0 < args.M) {
                         float4* dst = reinterpret_cast<float4*>(args.sk_partial) +
                                       (size_t)((int64_t)sg.t * args.split_k + sg.piece) * (C::ROWS * BN / 4) +
-                                      ((((size_t)q * C::HALVES + (ew >> 2)) * (C::EPI_COLS / 4) + c * 8) << 5) + lane;
+                                      ((((size_t)q * C::HALVES + (ew >> 2)) * (C::EPI_COLS / 4) + c * 8 + hh * 4) << 5) +
+                                      lane;
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
+                        for (int v = 0; v < 4; ++v)
                             __stcg(dst + v * 32,
                                    make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
                                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
                     }
-                    continue;
+                    return;
                 }
                 if (tail) {
-                    // Raw fp32 accumulator of this piece: row `lane`, columns c*32..+31.
+                    // Raw fp32 accumulator of this piece: row `lane`, columns c*32 + hh*16 ..+15.
 #pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        __stcg(my_part + (c * 8 + v) * 32,
+                    for (int v = 0; v < 4; ++v)
+                        __stcg(my_part + (c * 8 + hh * 4 + v) * 32,
                                make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
                                            __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
-                    continue;
+                    return;
                 }
                 if (head) {
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + pp[v].x);
-                        r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + pp[v].y);
-                        r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + pp[v].z);
-                        r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + pp[v].w);
-                    }
-                    // Next chunk's partial, in flight while this one is packed and stored.
-                    if (c + 1 < C::EPI_COLS / 32) {
-#pragma unroll
-                        for (int v = 0; v < 8; ++v) pp[v] = __ldcg(their_part + ((c + 1) * 8 + v) * 32);
+                    for (int v = 0; v < 4; ++v) {
+                        r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + pp[hh * 4 + v].x);
+                        r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + pp[hh * 4 + v].y);
+                        r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + pp[hh * 4 + v].z);
+                        r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + pp[hh * 4 + v].w);
                     }
                 }
-                uint32_t packed[16];
+                uint32_t packed[8];
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 w4 = *reinterpret_cast<const float4*>(sw_s + c * 32 + j);
-                    const float4 b4 = *reinterpret_cast<const float4*>(b_s + c * 32 + j);
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(sw_s + c * 32 + hh * 16 + j);
+                    const float4 b4 = *reinterpret_cast<const float4*>(b_s + c * 32 + hh * 16 + j);
                     const float o0 = fmaf(__uint_as_float(r[j + 0]) * sa, w4.x, b4.x);
                     const float o1 = fmaf(__uint_as_float(r[j + 1]) * sa, w4.y, b4.y);
                     const float o2 = fmaf(__uint_as_float(r[j + 2]) * sa, w4.z, b4.z);
@@ -820,18 +815,43 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                     packed[j / 2] = pack_bf16x2(o0, o1);
                     packed[j / 2 + 1] = pack_bf16x2(o2, o3);
                 }
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int phys = (hh * 2 + k) ^ ((lane >> 1) & 3);
+                    *reinterpret_cast<uint4*>(stg + lane * 64 + phys * 16) =
+                        make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+                }
+            };
+            // Chunks this warp holds (warp-uniform; fewer where the tile passes N).
+            const int base_n = tc.tn * BN + col0;
+            int nch = failed ? 0 : (n_tile - base_n + 31) / 32;
+            if (nch > C::EPI_COLS / 32) nch = C::EPI_COLS / 32;
+            if (nch < 0) nch = 0;
+            // Two 16-register buffers: the TMEM load of the next half is in
+            // flight while the current half is processed.
+            uint32_t ra[16], rb[16];
+            if (nch > 0) tmem_ld_32x32b_x16(t_addr, ra);
+#pragma unroll 1
+            for (int c = 0; c < nch; ++c) {
+                const int n0 = base_n + c * 32;
+                tmem_wait_ld16(ra);
+                tmem_ld_32x32b_x16(t_addr + c * 32 + 16, rb);
+                const bool store = !split && !tail;
                 // The single staging buffer is free once the previous store has read it.
-                if (stores >= 1) {
+                if (store && stores >= 1) {
                     if (lane == 0) bulk_wait_group_read<0>();
                     __syncwarp();
                 }
-                // Row `lane` of a 32 x 32 bf16 box, 64-byte rows, 64-byte swizzle.
+                half(c, 0, ra);
+                tmem_wait_ld16(rb);
+                if (c + 1 < nch) tmem_ld_32x32b_x16(t_addr + (c + 1) * 32, ra);
+                half(c, 1, rb);
+                if (head && c + 1 < C::EPI_COLS / 32) {
+                    // Next chunk's partial, in flight while this chunk is stored.
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const int phys = k4 ^ ((lane >> 1) & 3);
-                    *reinterpret_cast<uint4*>(stg + lane * 64 + phys * 16) =
-                        make_uint4(packed[4 * k4], packed[4 * k4 + 1], packed[4 * k4 + 2], packed[4 * k4 + 3]);
+                    for (int v = 0; v < 8; ++v) pp[v] = __ldcg(their_part + ((c + 1) * 8 + v) * 32);
                 }
+                if (!store) continue;
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0 && row0 < args.M) {
