@@ -80,6 +80,8 @@ def load_library():
     L.fp8_linear_workspace_size.argtypes = [p]
     L.fp8_linear_workspace_size.restype = ctypes.c_size_t
     L.fp8_linear_set_workspace.argtypes = [p, p, ctypes.c_size_t]
+    L.fp8_linear_workspace_flag_bytes.argtypes = [p]
+    L.fp8_linear_workspace_flag_bytes.restype = ctypes.c_size_t
     L.fp8_scaled_linear.argtypes = [p, i64, p, p, p, p, p, p, p]
     L.fp8_scaled_linear_multi.argtypes = [ctypes.POINTER(p), i32, i64, p, p, p, ctypes.POINTER(p), p]
     L.fp8_scaled_linear_noalloc.argtypes = [p, i64, p, p, p]
@@ -365,6 +367,11 @@ class FP8Linear:
         _check(L.fp8_linear_set_workspace(self._h, workspace.data_ptr(), workspace.numel() * workspace.element_size()))
         self.workspace = workspace  # keep it alive while attached
         return workspace
+
+    def workspace_flag_bytes(self) -> int:
+        """Bytes at the start of the workspace holding flags and counters (zero
+        after attaching and between launches)."""
+        return int(load_library().fp8_linear_workspace_flag_bytes(self._h))
 
     def detach_workspace(self) -> None:
         _check(load_library().fp8_linear_set_workspace(self._h, None, 0))

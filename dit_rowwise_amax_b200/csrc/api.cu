@@ -302,18 +302,19 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
             return unsupported("split-K plan exceeds the workspace");
         args.split_k = split;
         args.split_arrive = static_cast<uint32_t*>(hs[0]->sk_ws) + split_flag_offset_words(pairs);
-        args.sk_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(hs[0]->sk_ws) +
-                                                   (stream_k_workspace_bytes(pairs) -
-                                                    (size_t)pairs * kSkPartialBytesPerUnit));
+        args.sk_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(hs[0]->sk_ws) + sk_flag_area_bytes(pairs));
     }
     if (n == 1 && cfg == kCfgPair256 && hs[0]->sk_ws != nullptr && tiles >= units && num_kb >= kSkMinKBlocks) {
         const int64_t waves = (tiles + units - 1) / units;
         if ((waves * units - tiles) * 4 > waves * units) {
+            // units <= pairs: the layout is the one the workspace was sized for.
+            const int pairs = hs[0]->num_sms / 2;
+            uint8_t* ws = static_cast<uint8_t*>(hs[0]->sk_ws);
             args.stream_k = 1;
-            args.sk_flag = static_cast<uint32_t*>(hs[0]->sk_ws);
-            args.sk_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(hs[0]->sk_ws) +
-                                                       (stream_k_workspace_bytes(units) -
-                                                        (size_t)units * kSkPartialBytesPerUnit));
+            args.sk_flag = reinterpret_cast<uint32_t*>(ws);
+            args.sk_partial = reinterpret_cast<float*>(ws + sk_flag_area_bytes(pairs));
+            args.sk_partial_head =
+                reinterpret_cast<float*>(ws + sk_flag_area_bytes(pairs) + (size_t)pairs * kSkPartialBytesPerUnit);
         }
     }
     args.sa = sa;
@@ -490,6 +491,12 @@ size_t fp8_linear_workspace_size(fp8dit_linear h) {
     return stream_k_workspace_bytes(h->num_sms / 2);
 }
 
+size_t fp8_linear_workspace_flag_bytes(fp8dit_linear h) {
+    t_last_error[0] = 0;
+    if (!h) return 0;
+    return sk_flag_area_bytes(h->num_sms / 2);
+}
+
 fp8dit_status fp8_linear_set_workspace(fp8dit_linear h, void* workspace, size_t bytes) {
     t_last_error[0] = 0;
     if (!h) return invalid("null handle");
@@ -505,7 +512,7 @@ fp8dit_status fp8_linear_set_workspace(fp8dit_linear h, void* workspace, size_t 
     cudaError_t e = cudaGetDevice(&prev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (h->device != prev && (e = cudaSetDevice(h->device)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
-    e = cudaMemset(workspace, 0, need - (size_t)(h->num_sms / 2) * kSkPartialBytesPerUnit);  // the flags
+    e = cudaMemset(workspace, 0, sk_flag_area_bytes(h->num_sms / 2));  // the flags and counters
     if (h->device != prev) cudaSetDevice(prev);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace flags");
     h->sk_ws = workspace;

@@ -123,14 +123,15 @@ struct alignas(64) GemmArgs {
     int32_t qg_rows;       // rows per chunk (rows x K x 2 <= kQgBufBytes)
     int32_t qg_chunks;     // ceil(M / qg_rows)
     uint32_t* sk_flag;   // stream-K: [units + 1][2 CTAs][8 epilogue warps] (zero between launches)
+    float* sk_partial_head;  // stream-K: the heads' partials, laid out as the tails' in sk_partial
     float* sk_partial;   // stream-K: [units][2 CTAs][8 epilogue warps][32 rows][128 columns];
                          // split-K: [tiles][split_k][4 quarters][epilogue warps / 4 column parts]
                          //          [128 / (epilogue warps / 4) / 4 float4][32 rows]
 };
 
 // Stream-K / split-K workspace for `units` CTA pairs: a flag area, then the
-// partials. The flag area holds the stream-K flags ((units + 1) x 16 words,
-// indexed by the unit that finishes a tile and its successor), then the
+// partials. The flag area holds the stream-K marks ((units + 1) x 16 words,
+// indexed by the unit whose first segment ends a split tile), then the
 // split-K arrival counters (one per tile: a split launch has at most one tile
 // per pair; followed by `units` spare words), then the fused linear's
 // counters (2 + kQgMaxRowBlocks words). Every region starts zeroed by
@@ -162,9 +163,13 @@ constexpr int kSplitMinKBlocksTotalW8 = 32;  // the same for weight-only (64 bf1
 constexpr int kSplitMinKBlocks = 6;        // split-K: k-blocks per piece (one ring), at least
 constexpr int kSplitMaxPieces = 8;         // split-K: pieces per tile, at most
 constexpr size_t kSplitPieceBytes = 128 * 128 * sizeof(float);  // one fp32 128 x 128 partial
+inline size_t sk_flag_area_bytes(int units) {
+    return ((qg_offset_words(units) + 2 + kQgMaxRowBlocks) * sizeof(uint32_t) + 4095) & ~(size_t)4095;
+}
+// The flag area, then two partial areas of `units` x kSkPartialBytesPerUnit:
+// stream-K tails' partials (also split-K's), then stream-K heads' partials.
 inline size_t stream_k_workspace_bytes(int units) {
-    const size_t flags = ((qg_offset_words(units) + 2 + kQgMaxRowBlocks) * sizeof(uint32_t) + 4095) & ~(size_t)4095;
-    return flags + (size_t)units * kSkPartialBytesPerUnit;
+    return sk_flag_area_bytes(units) + 2 * (size_t)units * kSkPartialBytesPerUnit;
 }
 
 // Tile configurations the plan chooses from.

@@ -222,6 +222,11 @@ __device__ __forceinline__ bool wait_count_bounded(const uint32_t* p, uint32_t w
 __device__ __forceinline__ void red_add_release_gpu_u32(uint32_t* p, uint32_t v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t atom_exch_acq_rel_gpu_u32(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.exch.b32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
 __device__ __forceinline__ void st_release_gpu_u32(uint32_t* p, uint32_t v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -704,41 +709,47 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             // so every warp access moves 512 contiguous bytes.
             const bool tail = !split && sg.k0 > 0;
             const bool head = !split && sg.k0 == 0 && sg.k1 < args.num_kb;
+            // Stream-K: a tile split between units u (head: the tile's start, u's
+            // last segment) and u + 1 (tail: the tile's end, u + 1's first
+            // segment) is finished by whichever of the two warps arrives
+            // second, so neither ever waits for the other. Per epilogue warp
+            // one flag word F: 0 = nothing stored, 1 = the tail's partial is
+            // stored, 2 = the head's partial is stored. The tail stores its
+            // partial and swaps in 1; the head, if F already reads 1, finishes
+            // at once, else stores its own partial and swaps in 2. A swap that
+            // returns the other side's mark makes this warp the finisher: it
+            // adds the other partial to its own accumulator (fp32 addition
+            // commutes, so the result does not depend on which side finishes),
+            // applies the epilogue, stores y and clears F for the next launch.
             const size_t part_elems = 32 * C::EPI_COLS;
-            float4* my_part = nullptr;
-            const float4* their_part = nullptr;
+            uint32_t* sk_f = nullptr;
+            const float4* tail_part = nullptr;  // partials of the split tile this warp shares
+            const float4* head_part = nullptr;
             if (tail || head) {
-                const int slot = tail ? unit : unit + 1;  // tail: this unit's first segment
+                const int slot = tail ? unit : unit + 1;  // indexed by the tail's unit
                 const size_t idx = ((size_t)slot * 2 + rank) * C::EPI_WARPS + ew;
-                float* base = args.sk_partial + idx * part_elems;
-                if (tail) my_part = reinterpret_cast<float4*>(base) + lane;
-                else their_part = reinterpret_cast<const float4*>(base) + lane;
+                tail_part = reinterpret_cast<const float4*>(args.sk_partial + idx * part_elems) + lane;
+                head_part = reinterpret_cast<const float4*>(args.sk_partial_head + idx * part_elems) + lane;
+                sk_f = args.sk_flag + idx;
             }
-            float4 pp[8];  // the head's partial for the next column chunk
+            // Mode of the next pass over the accumulator: store it raw to
+            // `mine`, or add `theirs` (prefetched chunk by chunk into pp) and
+            // run the epilogue, or (neither) just the epilogue.
+            float4* mine = tail ? const_cast<float4*>(tail_part) : nullptr;
+            const float4* theirs = nullptr;
+            float4 pp[8];  // the other side's partial for the next column chunk
             if (head) {
-                // The partner unit wrote this partial in its first segment, long
-                // before this unit's last one; wait, bounded, for its flag, then
-                // fetch the first chunk while the accumulator is still being built.
-                const uint32_t* flag = args.sk_flag + ((size_t)(unit + 1) * 2 + rank) * C::EPI_WARPS + ew;
-                bool ok = ld_acquire_gpu_u32(flag) == 1u;
-                if (!ok) {
-                    const unsigned long long t0 = globaltimer_ns();
-                    while (!(ok = ld_acquire_gpu_u32(flag) == 1u)) {
-                        if (*abort_flag) break;
-                        if (globaltimer_ns() - t0 > args.err.limit_ns) {
-                            *abort_flag = 1;
-                            atomicOr(args.err.word, kDevErrTimeout);
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                }
-                if (!__all_sync(0xffffffffu, ok)) {
-                    if (lane == 0) abort_peer();
-                    break;
-                }
+                uint32_t f = 0;
+                if (lane == 0) f = ld_acquire_gpu_u32(sk_f);
+                f = __shfl_sync(0xffffffffu, f, 0);
+                __syncwarp();  // lane 0's acquire orders every lane's partial loads
+                if (f == 1u) {
+                    theirs = tail_part;  // the tail's partial is there: finish now
 #pragma unroll
-                for (int v = 0; v < 8; ++v) pp[v] = __ldcg(their_part + v * 32);
+                    for (int v = 0; v < 8; ++v) pp[v] = __ldcg(theirs + v * 32);
+                } else {
+                    mine = const_cast<float4*>(head_part);  // store ours; the tail may finish
+                }
             }
 
             // Every lane waits; the warp then agrees (and reconverges) before
@@ -763,10 +774,10 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             const int n_tile = args.prob[tc.g].N;
             const uint32_t t_addr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + col0;
             // One 16-column half of 32-column chunk c, its accumulator in r:
-            // split-K and stream-K tails store it raw; otherwise (a stream-K
-            // head first adds its partner's partial) scale, bias, bf16 and
-            // half of row `lane` of the chunk's 32 x 32 staging box (64-byte
-            // rows, 64-byte swizzle).
+            // split-K pieces and stream-K partials store it raw; otherwise (a
+            // stream-K finisher first adds the other side's partial) scale,
+            // bias, bf16 and half of row `lane` of the chunk's 32 x 32 staging
+            // box (64-byte rows, 64-byte swizzle).
             auto half = [&](int c, int hh, uint32_t(&r)[16]) {
                 if (split) {
                     // This piece's raw fp32 partial, [q][column part][float4][lane]:
@@ -785,16 +796,17 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                     }
                     return;
                 }
-                if (tail) {
-                    // Raw fp32 accumulator of this piece: row `lane`, columns c*32 + hh*16 ..+15.
+                if (mine != nullptr) {
+                    // Raw fp32 accumulator: row `lane`, columns c*32 + hh*16 ..+15,
+                    // lane-fastest (every warp store moves 512 contiguous bytes).
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
-                        __stcg(my_part + (c * 8 + hh * 4 + v) * 32,
+                        __stcg(mine + (c * 8 + hh * 4 + v) * 32,
                                make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
                                            __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
                     return;
                 }
-                if (head) {
+                if (theirs != nullptr) {
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + pp[hh * 4 + v].x);
@@ -829,6 +841,11 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             if (nch < 0) nch = 0;
             // Two 16-register buffers: the TMEM load of the next half is in
             // flight while the current half is processed.
+            // Pass 0 over the accumulator; a stream-K warp that learns after
+            // publishing its partial that it finishes the tile makes pass 1.
+            bool finish = false;
+#pragma unroll 1
+            for (int pass = 0; pass < 2; ++pass) {
             uint32_t ra[16], rb[16];
             if (nch > 0) tmem_ld_32x32b_x16(t_addr, ra);
 #pragma unroll 1
@@ -836,7 +853,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 const int n0 = base_n + c * 32;
                 tmem_wait_ld16(ra);
                 tmem_ld_32x32b_x16(t_addr + c * 32 + 16, rb);
-                const bool store = !split && !tail;
+                const bool store = !split && mine == nullptr;
                 // The single staging buffer is free once the previous store has read it.
                 if (store && stores >= 1) {
                     if (lane == 0) bulk_wait_group_read<0>();
@@ -846,10 +863,10 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 tmem_wait_ld16(rb);
                 if (c + 1 < nch) tmem_ld_32x32b_x16(t_addr + (c + 1) * 32, ra);
                 half(c, 1, rb);
-                if (head && c + 1 < C::EPI_COLS / 32) {
+                if (theirs != nullptr && c + 1 < C::EPI_COLS / 32) {
                     // Next chunk's partial, in flight while this chunk is stored.
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) pp[v] = __ldcg(their_part + ((c + 1) * 8 + v) * 32);
+                    for (int v = 0; v < 8; ++v) pp[v] = __ldcg(theirs + ((c + 1) * 8 + v) * 32);
                 }
                 if (!store) continue;
                 fence_proxy_async_smem();
@@ -860,19 +877,30 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 }
                 ++stores;
             }
-            if (tail) {
-                // Publish the partial: every lane's stores, then the flag.
-                __threadfence();
-                __syncwarp();
-                if (lane == 0)
-                    st_release_gpu_u32(args.sk_flag + ((size_t)unit * 2 + rank) * C::EPI_WARPS + ew, 1u);
+            if (pass == 1 || !(tail || head) || failed) break;
+            finish = theirs != nullptr;  // a head that found the tail's partial
+            if (mine == nullptr) break;
+            // Publish the partial (every lane's stores, then the mark) and
+            // learn whether the other side has already been here.
+            __threadfence();
+            __syncwarp();
+            uint32_t old = 0;
+            if (lane == 0) old = atom_exch_acq_rel_gpu_u32(sk_f, tail ? 1u : 2u);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            __syncwarp();  // lane 0's acquire orders every lane's partial loads
+            finish = old == (tail ? 2u : 1u);
+            if (!finish) break;
+            mine = nullptr;  // pass 1: add the other side's partial, epilogue, y
+            theirs = tail ? head_part : tail_part;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) pp[v] = __ldcg(theirs + v * 32);
             }
-            if (head) {
-                // Every lane has its partial in registers: clear the flag, so the
+            if (finish) {
+                // This warp finished the split tile: clear the mark, so the
                 // workspace is ready for the next launch without a host reset
-                // (stream-ordered launches, CUDA graph replays included).
+                // (stream-ordered launches and graph replays included).
                 __syncwarp();
-                if (lane == 0) args.sk_flag[((size_t)(unit + 1) * 2 + rank) * C::EPI_WARPS + ew] = 0u;
+                if (lane == 0) *sk_f = 0u;
             }
             tc_fence_before();
             __syncwarp();

@@ -192,13 +192,11 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  * tile-per-pair schedule (a nearly empty last wave: e.g. 150 tiles on 74
  * pairs) and a tile has at least 8 k-blocks of 128, each pair instead takes
  * an equal share of the layer's k-blocks; a tile split between two pairs is
- * finished by one of them after the other has stored its fp32 partial in this
- * workspace. Results stay deterministic (the two parts are added once, in
- * fp32) but differ in rounding from the plain schedule. The finishing pair
- * waits (bounded) for its partner's partial, which its partner computes
- * first, so the schedule relies on all of the launch's pairs running at the
- * same time: with other kernels holding SMs meanwhile, that wait may expire
- * (FP8DIT_ERR_TIMEOUT).
+ * finished by whichever of the two gets there second, from the fp32 partial
+ * the other has stored in this workspace; neither waits for the other, so the
+ * launch does not need all of its pairs resident at once. Results stay
+ * deterministic (the two parts are added once, in fp32, whichever side
+ * finishes) but differ in rounding from the plain schedule.
  * The same workspace enables split-K for few tiles and a long K: when the
  * 128 x 128 tiles of a small-M call fill at most half of the SMs and K has at
  * least 48 k-blocks of 128 (K >= 6144; e.g. text tokens through an FFN-down
@@ -212,7 +210,7 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  * 2048; K >= 4096 above 64 rows). fp8_scaled_linear_multi uses the workspace
  * of its first layer. Without a workspace, or for other shapes (the
  * FFN shapes among them), the plain schedule is used.
- *   fp8_linear_workspace_size: bytes needed on the layer's device (~19 MB on
+ *   fp8_linear_workspace_size: bytes needed on the layer's device (~38 MB on
  *     148 SMs), the same for every M.
  *   fp8_linear_set_workspace: attach caller-owned DEVICE memory (256-byte
  *     aligned, at least that size) or detach with NULL, while no call that
@@ -228,6 +226,9 @@ fp8dit_status fp8_linear_destroy(fp8dit_linear h);
  */
 size_t fp8_linear_workspace_size(fp8dit_linear h);
 fp8dit_status fp8_linear_set_workspace(fp8dit_linear h, void* workspace, size_t bytes);
+/* Bytes at the start of the workspace that hold its flags and counters: zero
+ * after attaching and between launches (the rest holds fp32 partials). */
+size_t fp8_linear_workspace_flag_bytes(fp8dit_linear h);
 
 /*
  * Forward of one FP8 linear layer ("从 BF16 到 FP8", sections 三.1, 三.3, 三.5):

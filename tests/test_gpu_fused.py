@@ -49,10 +49,9 @@ def check_rows(y, qa, sa, qw, sw, bias, rows):
 
 
 def counters_zero(layer):
-    ws = layer.workspace
-    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
-    flag_bytes = ws.numel() - pairs * 2 * 8 * 32 * 128 * 4  # everything before the fp32 partials
-    return int(torch.count_nonzero(ws[:flag_bytes])) == 0
+    flag_bytes = layer.workspace_flag_bytes()  # the flags and counters at the start of the workspace
+    assert 0 < flag_bytes < layer.workspace.numel()
+    return int(torch.count_nonzero(layer.workspace[:flag_bytes])) == 0
 
 
 @pytest.mark.parametrize("cfg", ["ffn_up", "ffn_down"])

@@ -280,8 +280,6 @@ def test_split_k_leaves_counters_cleared():
         layer.forward_weight_only(to_device_bf16(synth.normal_bf16(f"gpu/split/clr/A16{M}", (M, K), 1.0)))
     torch.cuda.synchronize()
     assert fp8.device_error() == 0
-    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
-    partial_bytes = pairs * 2 * 8 * 32 * 128 * 4  # the fp32 partial area after the flags
-    flag_bytes = ws.numel() - partial_bytes
-    assert flag_bytes > 0
+    flag_bytes = layer.workspace_flag_bytes()  # the flags and counters at the start of the workspace
+    assert 0 < flag_bytes < ws.numel()
     assert int(torch.count_nonzero(ws[:flag_bytes])) == 0

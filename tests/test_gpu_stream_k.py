@@ -111,3 +111,41 @@ def test_stream_k_cuda_graph_replays():
             torch.cuda.synchronize()
             assert fp8.device_error() == 0
             assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), f"replay {rep} differs"
+
+
+def test_stream_k_concurrent_launches_leave_marks_cleared():
+    """Stream-K launches of two layers (each with its own workspace) on two
+    streams at once, beside a pair-tile GEMM on a third: a split tile is
+    finished by whichever of its two units gets there second, so nothing
+    waits on a unit that has not started. Every output equals the same call
+    run alone, bit for bit; no device error; every mark is back at zero."""
+    M, N, K = 4864, 2048, 8192
+    d = synth.ffn_down()
+    layers, acts, refs = [], [], []
+    for i in range(2):
+        layer, _, _ = layer_and_codes(d["W"], synth.normal_bf16(f"gpu/sk/conc/b{i}", (N,), 0.1))
+        layer.attach_workspace()
+        qa, sa = fp8.quantize_rowwise(to_device_bf16(synth.normal_bf16(f"gpu/sk/conc/A{i}", (M, K), 1.0)))
+        layers.append(layer)
+        acts.append((qa, sa))
+        refs.append(layer.forward_fp8(qa, sa))
+    u = synth.ffn_up()
+    big = fp8.FP8Linear.from_weight(to_device_bf16(u["W"]), to_device_bf16(u["bias"]))
+    big_q = fp8.quantize_rowwise(to_device_bf16(u["A"]))
+    torch.cuda.synchronize()
+    assert fp8.device_error() == 0
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    outs = [[torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(6)] for _ in range(2)]
+    for it in range(6):
+        with torch.cuda.stream(streams[2]):
+            big.forward_fp8(*big_q)
+        for i in range(2):
+            with torch.cuda.stream(streams[i]):
+                layers[i].forward_fp8(*acts[i], y=outs[i][it])
+    torch.cuda.synchronize()
+    assert fp8.device_error() == 0
+    for i in range(2):
+        for it in range(6):
+            assert torch.equal(outs[i][it].view(torch.int16), refs[i].view(torch.int16)), (i, it)
+        nb = layers[i].workspace_flag_bytes()
+        assert int(torch.count_nonzero(layers[i].workspace[:nb])) == 0
