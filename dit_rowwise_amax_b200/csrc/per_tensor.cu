@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
         const bool is_amax = off < amax_chunks_here;
         const int t = is_amax ? j : j - 1;
         const int64_t chunk = is_amax ? off : off - amax_chunks_here;
-        const PerTensorDevDesc& d = a.d[t];
+        const PerTensorDevDesc d = a.d[t];  // a register copy: the loops below read it often
         const int64_t begin = chunk * kChunk;
         const int64_t end = min(d.numel, begin + kChunk);
 
