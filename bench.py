@@ -366,21 +366,6 @@ def main():
     if fp8.device_error(dev) != 0:
         raise RuntimeError("device error during warm-up")
 
-    # Per-kernel and per-layer regions: KR back-to-back launches (or layer
-    # calls) on the rotating buffers, captured in a CUDA graph and timed over
-    # one replay; consecutive launches overlap launch and tail as in the step,
-    # the graph takes the host's per-call launch cost (~8 us from Python) out
-    # of the shorter kernels' figures, and KR >= 200 amortises the region's
-    # first launch, which has no predecessor to overlap with. The HBM-bound
-    # quantisers go first, before tens of milliseconds of power-capped GEMMs.
-    KR = max(args.steps, 200)
-    k_avg = {}
-    for name, *_ in FFN:
-        k_avg[f"quantize_{name}"] = graph_region_ms(torch, lambda i, n=name: quantize(n, i), KR, dev, world)
-    peaks, peak_src = load_peaks()
-    extras = world == 1 and rank == 0 and not args.no_extras
-    q_hidden = measure_hidden_quantizer(fp8, torch, synth, dev, up, peaks["hbm_gbs"]) if extras else {}
-
     # Timed region 1 (the headline value): the K steps captured into one CUDA
     # graph (after the W eager warm-up steps), replayed once untimed to upload
     # and warm it, then once timed; only the region is bracketed by events, so
@@ -427,6 +412,21 @@ def main():
     torch.cuda.synchronize()
     eager_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
 
+    # Per-kernel and per-layer regions: KR back-to-back launches (or layer
+    # calls) on the rotating buffers, captured in a CUDA graph and timed over
+    # one replay; consecutive launches overlap launch and tail as in the step,
+    # the graph takes the host's per-call launch cost (~8 us from Python) out
+    # of the shorter kernels' figures, and KR >= 200 amortises the region's
+    # first launch, which has no predecessor to overlap with. The HBM-bound
+    # quantisers go first, before tens of milliseconds of power-capped GEMMs
+    # (the headline step above lasts a few milliseconds).
+    KR = max(args.steps, 200)
+    k_avg = {}
+    for name, *_ in FFN:
+        k_avg[f"quantize_{name}"] = graph_region_ms(torch, lambda i, n=name: quantize(n, i), KR, dev, world)
+    peaks, peak_src = load_peaks()
+    extras = world == 1 and rank == 0 and not args.no_extras
+    q_hidden = measure_hidden_quantizer(fp8, torch, synth, dev, up, peaks["hbm_gbs"]) if extras else {}
     for name, *_ in FFN:
         k_avg[f"gemm_{name}"] = graph_region_ms(torch, lambda i, n=name: gemm(n, i), KR, dev, world)
     # Each FFN layer as a whole (quantiser + GEMM per call), three regions per
