@@ -227,9 +227,6 @@ __device__ __forceinline__ uint32_t atom_exch_acq_rel_gpu_u32(uint32_t* p, uint3
     asm volatile("atom.acq_rel.gpu.global.exch.b32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
     return old;
 }
-__device__ __forceinline__ void st_release_gpu_u32(uint32_t* p, uint32_t v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -846,54 +843,54 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
             bool finish = false;
 #pragma unroll 1
             for (int pass = 0; pass < 2; ++pass) {
-            uint32_t ra[16], rb[16];
-            if (nch > 0) tmem_ld_32x32b_x16(t_addr, ra);
+                uint32_t ra[16], rb[16];
+                if (nch > 0) tmem_ld_32x32b_x16(t_addr, ra);
 #pragma unroll 1
-            for (int c = 0; c < nch; ++c) {
-                const int n0 = base_n + c * 32;
-                tmem_wait_ld16(ra);
-                tmem_ld_32x32b_x16(t_addr + c * 32 + 16, rb);
-                const bool store = !split && mine == nullptr;
-                // The single staging buffer is free once the previous store has read it.
-                if (store && stores >= 1) {
-                    if (lane == 0) bulk_wait_group_read<0>();
+                for (int c = 0; c < nch; ++c) {
+                    const int n0 = base_n + c * 32;
+                    tmem_wait_ld16(ra);
+                    tmem_ld_32x32b_x16(t_addr + c * 32 + 16, rb);
+                    const bool store = !split && mine == nullptr;
+                    // The single staging buffer is free once the previous store has read it.
+                    if (store && stores >= 1) {
+                        if (lane == 0) bulk_wait_group_read<0>();
+                        __syncwarp();
+                    }
+                    half(c, 0, ra);
+                    tmem_wait_ld16(rb);
+                    if (c + 1 < nch) tmem_ld_32x32b_x16(t_addr + (c + 1) * 32, ra);
+                    half(c, 1, rb);
+                    if (theirs != nullptr && c + 1 < C::EPI_COLS / 32) {
+                        // Next chunk's partial, in flight while this chunk is stored.
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) pp[v] = __ldcg(theirs + ((c + 1) * 8 + v) * 32);
+                    }
+                    if (!store) continue;
+                    fence_proxy_async_smem();
                     __syncwarp();
+                    if (lane == 0 && row0 < args.M) {
+                        tma_store_2d(&args.tmY[tc.g], stg, n0, row0);
+                        bulk_commit_group();
+                    }
+                    ++stores;
                 }
-                half(c, 0, ra);
-                tmem_wait_ld16(rb);
-                if (c + 1 < nch) tmem_ld_32x32b_x16(t_addr + (c + 1) * 32, ra);
-                half(c, 1, rb);
-                if (theirs != nullptr && c + 1 < C::EPI_COLS / 32) {
-                    // Next chunk's partial, in flight while this chunk is stored.
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) pp[v] = __ldcg(theirs + ((c + 1) * 8 + v) * 32);
-                }
-                if (!store) continue;
-                fence_proxy_async_smem();
+                if (pass == 1 || !(tail || head) || failed) break;
+                finish = theirs != nullptr;  // a head that found the tail's partial
+                if (mine == nullptr) break;
+                // Publish the partial (every lane's stores, then the mark) and
+                // learn whether the other side has already been here.
+                __threadfence();
                 __syncwarp();
-                if (lane == 0 && row0 < args.M) {
-                    tma_store_2d(&args.tmY[tc.g], stg, n0, row0);
-                    bulk_commit_group();
-                }
-                ++stores;
-            }
-            if (pass == 1 || !(tail || head) || failed) break;
-            finish = theirs != nullptr;  // a head that found the tail's partial
-            if (mine == nullptr) break;
-            // Publish the partial (every lane's stores, then the mark) and
-            // learn whether the other side has already been here.
-            __threadfence();
-            __syncwarp();
-            uint32_t old = 0;
-            if (lane == 0) old = atom_exch_acq_rel_gpu_u32(sk_f, tail ? 1u : 2u);
-            old = __shfl_sync(0xffffffffu, old, 0);
-            __syncwarp();  // lane 0's acquire orders every lane's partial loads
-            finish = old == (tail ? 2u : 1u);
-            if (!finish) break;
-            mine = nullptr;  // pass 1: add the other side's partial, epilogue, y
-            theirs = tail ? head_part : tail_part;
+                uint32_t old = 0;
+                if (lane == 0) old = atom_exch_acq_rel_gpu_u32(sk_f, tail ? 1u : 2u);
+                old = __shfl_sync(0xffffffffu, old, 0);
+                __syncwarp();  // lane 0's acquire orders every lane's partial loads
+                finish = old == (tail ? 2u : 1u);
+                if (!finish) break;
+                mine = nullptr;  // pass 1: add the other side's partial, epilogue, y
+                theirs = tail ? head_part : tail_part;
 #pragma unroll
-            for (int v = 0; v < 8; ++v) pp[v] = __ldcg(theirs + v * 32);
+                for (int v = 0; v < 8; ++v) pp[v] = __ldcg(theirs + v * 32);
             }
             if (finish) {
                 // This warp finished the split tile: clear the mark, so the
