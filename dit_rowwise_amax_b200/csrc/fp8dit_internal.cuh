@@ -141,12 +141,12 @@ struct alignas(64) GemmArgs {
 constexpr size_t kSkFlagBytesPerUnit = 2 * 8 * sizeof(uint32_t);
 inline size_t sk_flag_words(int units) { return (size_t)(units + 1) * 16; }
 inline size_t split_flag_offset_words(int units) { return sk_flag_words(units); }
-// Fused linear: rows are quantised in chunks staged in shared memory, a pool
-// of kQgBufs staging buffers of kQgBufBytes shared by the quantising warps;
+// Fused linear: rows are quantised in chunks staged in shared memory, one
+// staging buffer of kQgBufBytes per quantising warp (kQgBufs of them);
 // readiness is counted per 128-row block, so M <= 128 x kQgMaxRowBlocks;
 // rows up to kQgMaxK elements (one row must fit a buffer).
-constexpr int kQgBufs = 12;
-constexpr uint32_t kQgBufBytes = 16384;
+constexpr int kQgBufs = 8;
+constexpr uint32_t kQgBufBytes = 24576;
 constexpr int kQgClaim = 4;  // chunks claimed per atomic (even, >= 2)
 constexpr int kQgMaxRowBlocks = 8192;
 constexpr int kQgMaxK = 8192;

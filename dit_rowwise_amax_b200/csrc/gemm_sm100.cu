@@ -102,11 +102,11 @@ struct Cfg {
     static constexpr int STAGING_BYTES = EPI_WARPS * STG_BYTES;
     static constexpr int SWB_FLOATS = 2 * EPI_COLS;  // sw then bias as fp32, one copy per epilogue warp
     static constexpr int SWB_BYTES = EPI_WARPS * SWB_FLOATS * 4;
-    static constexpr int BAR_BYTES = 640;
+    static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_SMEM + STAGING_BYTES + SWB_BYTES + BAR_BYTES;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
     static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
-    static_assert((3 * STAGES + 2 * ACC + 2 + 2 * kQgBufs) * 8 + 4 * (8 + 2 * kQgBufs) <= BAR_BYTES, "barrier area");
+    static_assert((3 * STAGES + 2 * ACC + 2 + 2 * kQgBufs) * 8 + 4 * (6 + kQgBufs) <= BAR_BYTES, "barrier area");
     // Fused linear: kQgBufs chunks of bf16 rows (kQgBufBytes each) are staged
     // in the operand ring before the GEMM uses it.
     static_assert(!QG || kQgBufs * kQgBufBytes <= STAGES * STAGE_SMEM, "quantiser staging");
@@ -260,9 +260,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
     volatile uint32_t* split_fail = reinterpret_cast<volatile uint32_t*>(tmem_slot + 3);    // split-K
     volatile uint32_t* split_ok = reinterpret_cast<volatile uint32_t*>(tmem_slot + 4);      // split-K
     volatile int* qchunk = reinterpret_cast<volatile int*>(tmem_slot + 5);  // fused: chunk in each buffer [kQgBufs]
-    volatile int* qseq = qchunk + kQgBufs;                                  // fused: ticket of each buffer's use
-    volatile int* qticket = qseq + kQgBufs;                                 // fused: next ticket for the warps
-    volatile uint32_t* qlast = reinterpret_cast<volatile uint32_t*>(qticket + 1);  // fused: this CTA finished last
+    volatile uint32_t* qlast = tmem_slot + 5 + kQgBufs;  // fused: this CTA finished last
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -296,8 +294,6 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
         *split_ticket = 0u;
         *split_fail = 0u;
         *split_ok = 0u;
-        for (int b = 0; b < kQgBufs; ++b) qseq[b] = -1;
-        *qticket = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&args.tmA);
         for (int g = 0; g < args.G; ++g) {
@@ -329,45 +325,36 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
         // ------------------------------------------------ phase Q (fused linear)
         // Every CTA quantises rows of A until none are left unclaimed. Thread
         // 0 claims chunks of qg_rows rows in row order (kQgClaim chunks per
-        // atomic) and bulk-copies them in turn into a pool of kQgBufs staging
-        // buffers in the operand ring: this CTA's s-th chunk goes to buffer
-        // s mod kQgBufs once the chunk before it there has been handed back.
-        // The eight epilogue warps take the staged chunks in order (a ticket
-        // each from a shared counter), so a warp never waits for its own
-        // buffer to be refilled while others are full. A warp takes a chunk's
-        // rows one at a time: a sweep over the row in shared memory for its
-        // amax (shuffles), its scale, then a second sweep that writes its codes
-        // with the rowwise quantiser's arithmetic; it hands the buffer back,
-        // then counts the rows as done for their 128-row blocks (release). No
-        // warp waits for another warp's rows, and nothing here waits on
-        // another CTA; a chunk is only ever claimed by a running CTA, so every
-        // counted row block completes, and the GEMM below waits only for those
-        // counts.
-        // A staged buffer's use is identified by the ticket written into
-        // qseq[b] before its copy is issued: a warp holding ticket s first
-        // sees qseq[b] == s, which means use s / kQgBufs - 1 of the buffer has
-        // completed, and only then waits for the parity of use s / kQgBufs.
+        // atomic) and bulk-copies chunk i of this CTA into
+        // staging buffer i mod 8 in the operand ring. Quantising warp w owns
+        // buffer w: for each of its chunks it takes the rows one at a time, a
+        // sweep over the row in shared memory for its amax (shuffles), its
+        // scale, then a second sweep that writes its codes with the rowwise
+        // quantiser's arithmetic; after the chunk it counts the rows as done
+        // for their 128-row blocks (release) and hands the buffer back. No
+        // warp waits for another warp's rows and nothing here waits on another
+        // CTA; a chunk is only ever claimed by a running CTA, so every counted
+        // row block completes, and the GEMM below waits only for those counts.
         if (warp == 0 && lane == 0) {
             const int R = args.qg_rows;
+            // Chunks are claimed kQgClaim at a time; the next batch is claimed
+            // halfway through staging the current one, so the atomic's round
+            // trip overlaps the copies.
             int cur = (int)atomicAdd(args.qg_ctr, (uint32_t)kQgClaim);
             int nxt = 0;
             int k = 0;      // chunks of the current batch staged so far
-            int stop = 0;   // end marks given (one per quantising warp)
-            for (int s = 0; stop < 8; ++s) {
-                const int b = s % kQgBufs;
-                if (!mbar_wait_bounded(&qempty[b], (uint32_t)((s / kQgBufs) & 1) ^ 1u, abort_flag, args.err)) {
-                    *qticket = 0x40000000;  // give up: every later ticket finds an end mark
-                    for (int q = 0; q < kQgBufs; ++q) {
-                        qchunk[q] = -1;
-                        qseq[q] = -1;
-                    }
+            int stop = 0;   // buffers that have been given the end mark
+            for (int it = 0; stop < kQgBufs; ++it) {
+                const int b = it % kQgBufs;
+                if (!mbar_wait_bounded(&qempty[b], (uint32_t)((it / kQgBufs) & 1) ^ 1u, abort_flag, args.err)) {
+                    // Give up: mark every buffer, waiting for none of them.
+                    for (int q = 0; q < kQgBufs; ++q) qchunk[q] = -1;
+                    for (int q = 0; q < kQgBufs; ++q) mbar_arrive(&qfull[q]);
                     break;
                 }
                 const int c = cur + k;
                 if (c >= args.qg_chunks) {
-                    qchunk[b] = -1;  // no rows left: the warp holding ticket s stops
-                    __threadfence_block();
-                    qseq[b] = s;
+                    qchunk[b] = -1;  // no rows left: warp b stops at this buffer
                     mbar_arrive(&qfull[b]);
                     ++stop;
                     continue;
@@ -376,8 +363,6 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 const int rows = args.M - r0 < R ? args.M - r0 : R;
                 const uint32_t bytes = (uint32_t)rows * (uint32_t)args.K * 2u;
                 qchunk[b] = c;
-                __threadfence_block();
-                qseq[b] = s;
                 mbar_arrive_expect_tx(&qfull[b], bytes);
                 bulk_load_g2s(smem + (size_t)b * kQgBufBytes, args.qg_a + (size_t)r0 * args.K, bytes, &qfull[b]);
                 if (++k == kQgClaim / 2) nxt = (int)atomicAdd(args.qg_ctr, (uint32_t)kQgClaim);
@@ -387,40 +372,20 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                 }
             }
         } else if (warp >= 2) {
+            const int w = warp - 2;  // owns staging buffer w
             const int R = args.qg_rows;
             const int K = args.K;
             const int nvec = K >> 3;
-            while (true) {
-                int s = 0;
-                if (lane == 0) s = (int)atomicAdd(const_cast<uint32_t*>(reinterpret_cast<volatile uint32_t*>(qticket)), 1u);
-                s = __shfl_sync(0xffffffffu, s, 0);
-                const int b = s % kQgBufs;
-                // Wait (bounded) until the loader has issued use s of buffer b.
-                bool ok = true;
-                if (qseq[b] != s) {
-                    const unsigned long long t0 = globaltimer_ns();
-                    while (qseq[b] != s) {
-                        if (*abort_flag || globaltimer_ns() - t0 > args.err.limit_ns) {
-                            ok = false;
-                            break;
-                        }
-                    }
-                }
-                if (ok) ok = mbar_wait_bounded(&qfull[b], (uint32_t)((s / kQgBufs) & 1), abort_flag, args.err);
-                const int c = ok ? qchunk[b] : -1;
-                if (!__all_sync(0xffffffffu, c >= 0)) {
-                    if (lane == 0 && !ok && !*abort_flag) {
-                        *abort_flag = 1;
-                        atomicOr(args.err.word, kDevErrTimeout);
-                    }
-                    break;  // an end mark (or an expired wait)
-                }
+            for (int j = 0;; ++j) {
+                const bool ok = mbar_wait_bounded(&qfull[w], (uint32_t)(j & 1), abort_flag, args.err);
+                const int c = ok ? qchunk[w] : -1;
+                if (!__all_sync(0xffffffffu, c >= 0)) break;  // no more rows (or an expired wait)
                 const int r0 = c * R;
                 const int rows = args.M - r0 < R ? args.M - r0 : R;
                 for (int lr = 0; lr < rows; ++lr) {
                     const int64_t row = (int64_t)r0 + lr;
                     const uint4* src =
-                        reinterpret_cast<const uint4*>(smem + (size_t)b * kQgBufBytes + (size_t)lr * K * 2);
+                        reinterpret_cast<const uint4*>(smem + (size_t)w * kQgBufBytes + (size_t)lr * K * 2);
                     uint32_t packed = 0;
 #pragma unroll 4
                     for (int vi = lane; vi < nvec; vi += 32) packed = absmax8(src[vi], packed);
@@ -438,13 +403,11 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                     }
                     if (lane == 0) args.qg_s[row] = sc.s;
                 }
-                // The staged rows have been read (generic proxy): the buffer
-                // goes back before the copy engine (async proxy) refills it.
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&qempty[b]);
-                // The chunk's codes and scales, then its counts.
+                // The chunk's codes and scales, then its counts; the staged rows
+                // have been read (generic proxy) before the copy engine (async
+                // proxy) refills the buffer.
                 __threadfence();
+                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
                     for (int r = r0; r < r0 + rows;) {
@@ -453,6 +416,7 @@ __global__ void __launch_bounds__(Cfg<CG, BN, OPS>::THREADS, 1)
                         red_add_release_gpu_u32(args.qg_ctr + 2 + blk, (uint32_t)(e - r));
                         r = e;
                     }
+                    mbar_arrive(&qempty[w]);
                 }
             }
         }
