@@ -64,7 +64,7 @@ __device__ __forceinline__ float abs_bits_to_float(uint32_t bits) {
 
 // |x| bits of element e (tails).
 template <int SRC>
-__device__ __forceinline__ uint32_t abs_bits1(const void* src, int64_t e) {
+__device__ __forceinline__ uint32_t abs_bits1(const void* src, int e) {
     if constexpr (SRC == FP8DIT_SRC_F32) return __float_as_uint(static_cast<const float*>(src)[e]) & 0x7fffffffu;
     else return (uint32_t)static_cast<const uint16_t*>(src)[e] & 0x7fffu;
 }
@@ -121,7 +121,7 @@ __device__ __forceinline__ uint2 quant_vec_div(const uint4& v, float s) {
 
 // One element -> its code (tails), for any source type.
 template <int SRC, int FMT>
-__device__ __forceinline__ uint8_t quant1_any(const void* src, int64_t e, const ScaleCtx& c) {
+__device__ __forceinline__ uint8_t quant1_any(const void* src, int e, const ScaleCtx& c) {
     if constexpr (SRC == FP8DIT_SRC_BF16) {
         return quant1<FMT>(static_cast<const uint16_t*>(src)[e], c);
     } else {
@@ -139,63 +139,62 @@ __device__ __forceinline__ uint8_t quant1_any(const void* src, int64_t e, const 
     }
 }
 
-// Thread's share of the amax of chunk [begin, end) of a tensor, as |x| bits.
+// Thread's share of the amax of a chunk of n (<= kChunk) elements starting
+// at base, as |x| bits. In-chunk indices are 32-bit.
 template <int SRC>
-__device__ __forceinline__ uint32_t amax_chunk(const PerTensorDevDesc& d, int64_t begin, int64_t end) {
+__device__ __forceinline__ uint32_t amax_chunk(const void* base, int n) {
     constexpr int EPV = Src<SRC>::kEpv;
     constexpr int VPT = (int)(kChunk / EPV / kThreads);
-    const int64_t nvec = (end - begin) / EPV;  // whole vectors in this chunk
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(d.src) +
-                                                      begin * (SRC == FP8DIT_SRC_F32 ? 4 : 2));
+    const int nvec = n / EPV;  // whole vectors in this chunk
+    const uint4* src = static_cast<const uint4*>(base);
     uint32_t packed = 0;
 #pragma unroll 4
     for (int i = 0; i < VPT; ++i) {
-        const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+        const int vi = i * kThreads + (int)threadIdx.x;
         if (vi < nvec) packed = absmax_vec<SRC>(__ldg(src + vi), packed);
     }
     uint32_t m = SRC == FP8DIT_SRC_F32 ? packed : fold_halves(packed);
-    for (int64_t e = begin + nvec * EPV + threadIdx.x; e < end; e += kThreads) m = max(m, abs_bits1<SRC>(d.src, e));
+    for (int e = nvec * EPV + (int)threadIdx.x; e < n; e += kThreads) m = max(m, abs_bits1<SRC>(base, e));
     return m;
 }
 
-// Codes of chunk [begin, end) of a tensor with scale context c.
+// Codes of a chunk of n (<= kChunk) elements from base into dst, with scale
+// context c.
 template <int SRC, int FMT>
-__device__ __forceinline__ void quant_chunk(const PerTensorDevDesc& d, int64_t begin, int64_t end, const ScaleCtx& c) {
+__device__ __forceinline__ void quant_chunk(const void* base, uint8_t* dst, int n, const ScaleCtx& c) {
     constexpr int EPV = Src<SRC>::kEpv;
     constexpr int VPT = (int)(kChunk / EPV / kThreads);
-    const int64_t nvec = (end - begin) / EPV;
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(d.src) +
-                                                      begin * (SRC == FP8DIT_SRC_F32 ? 4 : 2));
-    uint8_t* dst = d.dst + begin;
+    const int nvec = n / EPV;
+    const uint4* src = static_cast<const uint4*>(base);
     if constexpr (SRC == FP8DIT_SRC_BF16) {
         const Quot2 q2 = quot2_of(c);
         if (c.fast) {
 #pragma unroll 4
             for (int i = 0; i < VPT; ++i) {
-                const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+                const int vi = i * kThreads + (int)threadIdx.x;
                 if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT, true>(__ldcs(src + vi), q2));
             }
         } else {
 #pragma unroll 4
             for (int i = 0; i < VPT; ++i) {
-                const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+                const int vi = i * kThreads + (int)threadIdx.x;
                 if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant8<FMT, false>(__ldcs(src + vi), q2));
             }
         }
     } else if constexpr (SRC == FP8DIT_SRC_F16) {
 #pragma unroll 4
         for (int i = 0; i < VPT; ++i) {
-            const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+            const int vi = i * kThreads + (int)threadIdx.x;
             if (vi < nvec) __stcs(reinterpret_cast<uint2*>(dst) + vi, quant_vec_div<SRC, FMT>(__ldcs(src + vi), c.s));
         }
     } else {
 #pragma unroll 4
         for (int i = 0; i < VPT; ++i) {
-            const int64_t vi = (int64_t)i * kThreads + threadIdx.x;
+            const int vi = i * kThreads + (int)threadIdx.x;
             if (vi < nvec) __stcs(reinterpret_cast<uint32_t*>(dst) + vi, quant_vec_div<SRC, FMT>(__ldcs(src + vi), c.s).x);
         }
     }
-    for (int64_t e = begin + nvec * EPV + threadIdx.x; e < end; e += kThreads) d.dst[e] = quant1_any<SRC, FMT>(d.src, e, c);
+    for (int e = nvec * EPV + (int)threadIdx.x; e < n; e += kThreads) dst[e] = quant1_any<SRC, FMT>(base, e, c);
 }
 
 template <int FMT>
@@ -225,15 +224,18 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
         const bool is_amax = off < amax_chunks_here;
         const int t = is_amax ? j : j - 1;
         const int64_t chunk = is_amax ? off : off - amax_chunks_here;
-        const PerTensorDevDesc d = a.d[t];  // a register copy: the loops below read it often
+        // Per item only the chunk's pointers, its length and the dtype stay
+        // live through the loops (32-bit in-chunk indices).
+        const PerTensorDevDesc& d = a.d[t];
+        const int src_dtype = d.src_dtype;  // uniform across the block (one tensor per item)
         const int64_t begin = chunk * kChunk;
-        const int64_t end = min(d.numel, begin + kChunk);
+        const int n = (int)min((int64_t)kChunk, d.numel - begin);
+        const void* base = static_cast<const uint8_t*>(d.src) + begin * (src_dtype == FP8DIT_SRC_F32 ? 4 : 2);
 
         if (is_amax) {
-            // The dtype is uniform across the block (one tensor per item).
-            uint32_t m = d.src_dtype == FP8DIT_SRC_F32   ? amax_chunk<FP8DIT_SRC_F32>(d, begin, end)
-                         : d.src_dtype == FP8DIT_SRC_F16 ? amax_chunk<FP8DIT_SRC_F16>(d, begin, end)
-                                                         : amax_chunk<FP8DIT_SRC_BF16>(d, begin, end);
+            uint32_t m = src_dtype == FP8DIT_SRC_F32   ? amax_chunk<FP8DIT_SRC_F32>(base, n)
+                         : src_dtype == FP8DIT_SRC_F16 ? amax_chunk<FP8DIT_SRC_F16>(base, n)
+                                                       : amax_chunk<FP8DIT_SRC_BF16>(base, n);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
             if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
@@ -264,9 +266,9 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
                     }
                 }
                 const uint32_t bits = ld_acquire_gpu(&a.amax_bits[t]);
-                const float amax = d.src_dtype == FP8DIT_SRC_F32   ? abs_bits_to_float<FP8DIT_SRC_F32>(bits)
-                                   : d.src_dtype == FP8DIT_SRC_F16 ? abs_bits_to_float<FP8DIT_SRC_F16>(bits)
-                                                                   : abs_bits_to_float<FP8DIT_SRC_BF16>(bits);
+                const float amax = src_dtype == FP8DIT_SRC_F32   ? abs_bits_to_float<FP8DIT_SRC_F32>(bits)
+                                   : src_dtype == FP8DIT_SRC_F16 ? abs_bits_to_float<FP8DIT_SRC_F16>(bits)
+                                                                 : abs_bits_to_float<FP8DIT_SRC_BF16>(bits);
                 s_amax = amax;
                 s_ok = ok;
                 if (ok && chunk == 0) *d.scale = scale_ctx<FMT>(amax).s;
@@ -274,9 +276,10 @@ __global__ void __launch_bounds__(kThreads) per_tensor_kernel(const __grid_const
             __syncthreads();
             if (s_ok) {
                 const ScaleCtx c = scale_ctx<FMT>(s_amax);
-                if (d.src_dtype == FP8DIT_SRC_F32) quant_chunk<FP8DIT_SRC_F32, FMT>(d, begin, end, c);
-                else if (d.src_dtype == FP8DIT_SRC_F16) quant_chunk<FP8DIT_SRC_F16, FMT>(d, begin, end, c);
-                else quant_chunk<FP8DIT_SRC_BF16, FMT>(d, begin, end, c);
+                uint8_t* dst = d.dst + begin;
+                if (src_dtype == FP8DIT_SRC_F32) quant_chunk<FP8DIT_SRC_F32, FMT>(base, dst, n, c);
+                else if (src_dtype == FP8DIT_SRC_F16) quant_chunk<FP8DIT_SRC_F16, FMT>(base, dst, n, c);
+                else quant_chunk<FP8DIT_SRC_BF16, FMT>(base, dst, n, c);
             }
         }
         __syncthreads();  // s_item / s_red / s_amax are rewritten next iteration
@@ -319,11 +322,19 @@ cudaError_t launch_per_tensor(const fp8dit_tensor_desc* host_descs, int32_t n, i
         args.stage_start[nb + 1] = pos;
         cudaError_t e = cudaMemsetAsync(ws, 0, per_tensor_workspace_bytes(nb), stream);
         if (e != cudaSuccess) return e;
-        const int64_t grid = std::min<int64_t>((int64_t)dev->num_sms * 8, total_chunks * 2);
-        if (fmt == FP8DIT_E4M3FN)
-            per_tensor_kernel<FP8DIT_E4M3FN><<<(unsigned)grid, kThreads, 0, stream>>>(args);
-        else
-            per_tensor_kernel<FP8DIT_E5M2><<<(unsigned)grid, kThreads, 0, stream>>>(args);
+        // A persistent grid: as many blocks as are resident at once (blocks
+        // beyond that would only start once the queue is drained).
+        void (*kernel)(PerTensorArgs) =
+            fmt == FP8DIT_E4M3FN ? per_tensor_kernel<FP8DIT_E4M3FN> : per_tensor_kernel<FP8DIT_E5M2>;
+        static int per_sm[2] = {0, 0};  // resident blocks per SM, per format (same on every sm_100a device)
+        int& resident = per_sm[fmt == FP8DIT_E4M3FN ? 0 : 1];
+        if (resident == 0) {
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kernel, kThreads, 0);
+            if (e != cudaSuccess) return e;
+            if (resident < 1) resident = 1;
+        }
+        const int64_t grid = std::min<int64_t>((int64_t)dev->num_sms * resident, total_chunks * 2);
+        kernel<<<(unsigned)grid, kThreads, 0, stream>>>(args);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
