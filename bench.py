@@ -429,11 +429,11 @@ def main():
     q_hidden = measure_hidden_quantizer(fp8, torch, synth, dev, up, peaks["hbm_gbs"]) if extras else {}
     for name, *_ in FFN:
         k_avg[f"gemm_{name}"] = graph_region_ms(torch, lambda i, n=name: gemm(n, i), KR, dev, world)
-    # Each FFN layer as a whole (quantiser + GEMM per call), three regions per
+    # Each FFN layer as a whole (quantiser + GEMM per call), five regions per
     # layer interleaved, the median kept: a region of 200 calls lasts 12-14 ms
     # and can land in a transient lower power state of the GPU.
     layer_runs = {name: [] for name, *_ in FFN}
-    for _ in range(3):
+    for _ in range(5):
         for name, *_ in FFN:
             layer_runs[name].append(graph_region_ms(torch, lambda i, n=name: linear(n, i), KR, dev, world))
     layer_ms = {name: statistics.median(v) for name, v in layer_runs.items()}
