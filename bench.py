@@ -50,6 +50,14 @@ FLOPS_PER_STEP = sum(2.0 * M * N * K for _, M, N, K in FFN)
 QBYTES = {name: 2 * M * K + M * K + 4 * M for name, M, N, K in FFN}
 FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Idle time before each per-kernel / per-layer region, so that every burst
+# figure starts from the same power state as the headline step. Right after
+# tens of milliseconds of power-capped GEMMs the power controller holds the
+# clocks down for a while: measured on one box, the FFN-up quantiser region
+# read 6.2 us and the FFN-down linear region 78 us straight after 27 ms of
+# FFN steps, and 5.1 / 69.5 us after 50 ms or more of idle. The loaded state
+# is reported separately (targets.sustained).
+REST_S = 0.2
 
 
 def config_dict(n_gpus: int) -> dict:
@@ -417,9 +425,8 @@ def main():
     # one replay; consecutive launches overlap launch and tail as in the step,
     # the graph takes the host's per-call launch cost (~8 us from Python) out
     # of the shorter kernels' figures, and KR >= 200 amortises the region's
-    # first launch, which has no predecessor to overlap with. The HBM-bound
-    # quantisers go first, before tens of milliseconds of power-capped GEMMs
-    # (the headline step above lasts a few milliseconds).
+    # first launch, which has no predecessor to overlap with. Every region
+    # starts after REST_S of idle (see REST_S).
     KR = max(args.steps, 200)
     k_avg = {}
     for name, *_ in FFN:
@@ -430,8 +437,7 @@ def main():
     for name, *_ in FFN:
         k_avg[f"gemm_{name}"] = graph_region_ms(torch, lambda i, n=name: gemm(n, i), KR, dev, world)
     # Each FFN layer as a whole (quantiser + GEMM per call), five regions per
-    # layer interleaved, the median kept: a region of 200 calls lasts 12-14 ms
-    # and can land in a transient lower power state of the GPU.
+    # layer interleaved, the median kept.
     layer_runs = {name: [] for name, *_ in FFN}
     for _ in range(5):
         for name, *_ in FFN:
@@ -608,11 +614,19 @@ def measure_e2e(fp8, torch, layers, host, dev, args, world):
                    f"{E2E_SLOTS} slots, copy-in / quantise + GEMM / copy-out overlapped) from pinned host memory"}
 
 
+def rest(torch):
+    """Let the GPU idle for REST_S before a burst region."""
+    torch.cuda.synchronize()
+    time.sleep(REST_S)
+
+
 def graph_region_ms(torch, fn, n, dev, world=1, warm=3):
     """Device time per call of n back-to-back calls of fn, captured into one
     CUDA graph and replayed (once untimed, to upload and warm it; then once
-    timed, events at the ends; max over ranks). Replaying removes the host's
-    per-call launch cost, which exceeds the device time of the smaller kernels."""
+    timed, events at the ends; max over ranks), after REST_S of idle.
+    Replaying removes the host's per-call launch cost, which exceeds the
+    device time of the smaller kernels."""
+    rest(torch)
     cur = torch.cuda.current_stream(dev)
     side = torch.cuda.Stream(dev)
     side.wait_stream(cur)
@@ -642,6 +656,8 @@ def graph_region_ms(torch, fn, n, dev, world=1, warm=3):
 
 
 def time_region(torch, fn, iters, dev, warm=3):
+    """Device time per call of iters eager calls of fn, after REST_S of idle."""
+    rest(torch)
     stream = torch.cuda.current_stream(dev)
     for i in range(warm):
         fn(i)
