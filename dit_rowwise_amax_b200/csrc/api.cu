@@ -331,7 +331,6 @@ static fp8dit_status run_gemm(const fp8dit_linear* hs, int32_t n, int64_t M, con
     args.M = (int32_t)M;
     args.K = (int32_t)hs[0]->K;
     args.G = n;
-    args.tiles_m = tiles_m;
     args.num_tiles = tiles;
     args.num_kb = (int32_t)num_kb;
     args.err = dev_err(dev);

@@ -91,7 +91,6 @@ struct alignas(64) GemmArgs {
     GemmProblem prob[kMaxGroups];
     const float* sa;
     int32_t M, K, G;
-    int32_t tiles_m;
     int32_t num_tiles;
     int32_t num_kb;
     DevErr err;
